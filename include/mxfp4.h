@@ -1,0 +1,155 @@
+/*
+ * mxfp4.h -- C ABI of the B200 (sm_100a) MXFP4 quantize / MoE expert-MLP library.
+ *
+ * MXFP4: every element is an E2M1 4-bit float (1 sign, 2 exponent, 1 mantissa bit)
+ * and each block of 32 consecutive elements shares one scale (agentlenshq.com,
+ * "Transformers 4.40 performance upgrades for OpenAI GPT-OSS: zero-build kernels,
+ * MXFP4 quantization, parallelism, and faster loading", section "What MXFP4 Is").
+ * The MoE expert MLP on MXFP4 expert weights is the layer that page runs through
+ * its downloadable MoE kernel (section "Zero-Build Kernels from the Hub").
+ *
+ * Encoding used throughout (the pages leave these open):
+ *   - E2M1 with exponent bias 1: magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6};
+ *     a 4-bit code is (sign << 3) | magnitude index;
+ *   - one E8M0 scale byte S per block, value 2^(S-127), S = 0xFF is NaN;
+ *   - packed codes: uint8 [rows, cols/2], element 2j in the low nibble of byte j;
+ *   - scales: uint8 [rows, cols/32], row-major; blocks run along the last
+ *     (contiguous) dimension, which for weights is the contraction dimension K.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps them.  Row-major, densely packed.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream).  Nothing synchronizes except
+ *     mxfp4_get_device_status().
+ *   - Arguments are validated on the host before anything is launched; an invalid
+ *     call launches nothing and returns a status.  Functions never print, abort
+ *     or exit.  A failed launch returns MXFP4_ERR_CUDA and the cudaError_t is kept
+ *     per host thread (mxfp4_last_cuda_error()).
+ *   - Kernels that wait on barriers do so with a time limit; on expiry they record
+ *     MXFP4_ERR_TIMEOUT in a per-device status word, clean up and return.  Read it
+ *     with mxfp4_get_device_status().
+ *   - The device must be compute capability 10.0 (B200, sm_100a), else MXFP4_ERR_ARCH.
+ *   - Pointers must be 16-byte aligned (MXFP4_ERR_MISALIGNED).
+ */
+#ifndef MXFP4_H_
+#define MXFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MXFP4_API __attribute__((visibility("default")))
+#else
+#define MXFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXFP4_OK = 0,
+    MXFP4_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size, bad enum   */
+    MXFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a dimension violates the stated multiples   */
+    MXFP4_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned            */
+    MXFP4_ERR_ARCH = 4,              /* current device is not sm_100                */
+    MXFP4_ERR_WORKSPACE = 5,         /* workspace missing or smaller than required  */
+    MXFP4_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed           */
+    MXFP4_ERR_TIMEOUT = 7            /* a device-side wait ran out of time          */
+} mxfp4_status;
+
+typedef enum { MXFP4_IN_BF16 = 0, MXFP4_IN_F32 = 1 } mxfp4_in_dtype;
+
+/* Block scale exponent s (scale = 2^s):
+ *   FLOOR: s = floor(log2(amax)) - 2 (OCP MX rule; |v|/2^s in (6, 8) saturates to 6);
+ *   CEIL:  smallest s with amax / 2^s <= 6 (never saturates).
+ * s is clamped to [-127, 127]; an all-zero block gets S = 0. */
+typedef enum { MXFP4_SCALE_FLOOR = 0, MXFP4_SCALE_CEIL = 1 } mxfp4_scale_rule;
+
+/* W4A16: bf16 activations x dequantized (bf16) MXFP4 weights, fp32 accumulation
+ *        on tcgen05 kind::f16.
+ * W4A4:  activations are MXFP4-quantized too (FLOOR rule, blocks along K) and the
+ *        product runs on the block-scaled tcgen05 kind::mxf4 MMA. */
+typedef enum { MXFP4_W4A16 = 0, MXFP4_W4A4 = 1 } mxfp4_mode;
+
+/* ---------------------------------------------------------------- quantize
+ * x [rows, cols] (bf16 or fp32 per `dt`) -> codes uint8 [rows, cols/2] and
+ * scales uint8 [rows, cols/32].  Per 32-element block: amax, E8M0 scale (rule),
+ * E2M1 round-to-nearest-even of |v|/2^s saturating at 6, input sign bit copied
+ * (-0 gives code 8); a block containing Inf/NaN gets S = 0xFF and zero codes.
+ * Requires cols % 32 == 0.  Bit-exact: exactly one correct output exists. */
+MXFP4_API mxfp4_status mxfp4_quantize(const void* x, mxfp4_in_dtype dt, int64_t rows, int64_t cols,
+                            uint8_t* codes, uint8_t* scales, mxfp4_scale_rule rule,
+                            void* stream);
+
+/* ---------------------------------------------------------------- dequantize
+ * codes uint8 [rows, cols/2] + scales uint8 [rows, cols/32] -> out bf16 [rows, cols].
+ * value = code_value * 2^(S-127) rounded once to bf16 (exact except overflow to
+ * Inf); S = 0xFF gives NaN.  Requires cols % 32 == 0. */
+MXFP4_API mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
+                              int64_t rows, int64_t cols, void* out_bf16, void* stream);
+
+/* ---------------------------------------------------------------- GEMM
+ * y [M, N] bf16 = x [M, K] bf16 . dequant(W)^T, W = MXFP4 codes [N, K/2] +
+ * scales [N, K/32]; fp32 accumulation, one rounding to bf16 at the end.
+ * Requires K % 64 == 0; any M >= 1, N >= 1.  Workspace: W4A16 needs none
+ * (ws may be NULL); W4A4 needs mxfp4_gemm_workspace_size() bytes (the quantized x). */
+MXFP4_API mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K,
+                        const uint8_t* w_codes, const uint8_t* w_scales, int64_t N,
+                        void* y_bf16, mxfp4_mode mode, void* ws, size_t ws_bytes,
+                        void* stream);
+MXFP4_API size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp4_mode mode);
+
+/* ---------------------------------------------------------------- routing
+ * Per token t of router logits [T, E] fp32: the top_k experts ordered by
+ * (logit descending, expert id ascending) -> ids int32 [T, top_k]; softmax over
+ * those k logits in fp32 -> weights fp32 [T, top_k]; then the pairs p = t*top_k + j
+ * grouped by expert: counts int32 [E], offsets int32 [E+1] (exclusive prefix
+ * sum), perm int32 [P] (perm[offsets[e] + r] = the r-th pair routed to e in
+ * ascending p) and inv int32 [P] (inv[perm[i]] = i), P = T*top_k.
+ * Requires 1 <= top_k <= min(E, 8), E <= 256, T*top_k < 2^31.
+ * ids/counts/offsets/perm/inv are bit-exact; weights match an fp64 softmax to
+ * ~1e-6 relative. */
+MXFP4_API mxfp4_status moe_mxfp4_route(const float* router_logits, int64_t T, int64_t E, int32_t top_k,
+                             int32_t* ids, float* weights, int32_t* counts, int32_t* offsets,
+                             int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
+                             void* stream);
+/* Scratch bytes moe_mxfp4_route needs in `ws` (per-chunk counts and ranks). */
+MXFP4_API size_t moe_mxfp4_route_workspace_size(int64_t T, int64_t E, int32_t top_k);
+
+/* ---------------------------------------------------------------- MoE expert MLP
+ * gpt-oss-style MoE expert MLP with MXFP4 expert weights, one layer:
+ *   route (as moe_mxfp4_route) -> gather x rows per expert ->
+ *   [g | u] = x . W13[e]^T   (W13 [E, 2I, H]: rows [0, I) gate, [I, 2I) up) ->
+ *   h = bf16( SiLU(g) * u )  (SiLU(g) = g / (1 + e^-g), fp32) ->
+ *   y = w_tj * (h . W2[e]^T) (W2 [E, H, I], weight applied in fp32) ->
+ *   out[t] = bf16( sum_j y_tj ) in slot order (deterministic; no atomics).
+ * x bf16 [T, H]; router_logits fp32 [T, E]; w13 codes uint8 [E, 2I, H/2] +
+ * scales uint8 [E, 2I, H/32]; w2 codes uint8 [E, H, I/2] + scales [E, H, I/32];
+ * out bf16 [T, H].  Requires H % 64 == 0, I % 64 == 0, 1 <= top_k <= min(E, 8),
+ * E <= 256, T*top_k < 2^31.  ws must hold moe_mxfp4_workspace_size() bytes
+ * (routing tables and the per-pair activations h / y). */
+MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,
+                           const float* router_logits, int64_t E, int32_t top_k,
+                           const uint8_t* w13_codes, const uint8_t* w13_scales, int64_t I,
+                           const uint8_t* w2_codes, const uint8_t* w2_scales,
+                           void* out_bf16, mxfp4_mode mode, void* ws, size_t ws_bytes,
+                           void* stream);
+MXFP4_API size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k,
+                                mxfp4_mode mode);
+
+/* ---------------------------------------------------------------- status
+ * Synchronizes `stream`, then returns and clears the current device's device-side
+ * status word (MXFP4_OK, or MXFP4_ERR_TIMEOUT if a kernel gave up waiting).
+ * Returns MXFP4_ERR_CUDA if the synchronization itself failed. */
+MXFP4_API mxfp4_status mxfp4_get_device_status(void* stream);
+/* cudaError_t of the last failed CUDA call on this host thread (0 if none). */
+MXFP4_API int mxfp4_last_cuda_error(void);
+/* Static, human-readable name of a status code. */
+MXFP4_API const char* mxfp4_status_string(mxfp4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXFP4_H_ */

@@ -1,0 +1,153 @@
+"""MXFP4 quantization and the MXFP4-weight MoE expert MLP on NVIDIA B200 (sm_100a).
+
+Python face of the C-ABI library ``libmxfp4.so`` (``include/mxfp4.h``).  The
+functions below carry the C entry points' names and only marshal arguments:
+torch tensors provide device memory and the current CUDA stream, and every step
+runs in the library's CUDA kernels.  There is no CPU or fallback path: if the
+library is missing, calls raise ``Mxfp4LibraryMissing``.
+
+MXFP4 = E2M1 4-bit codes (1 sign, 2 exponent, 1 mantissa bit) with one E8M0
+power-of-two scale per 32 consecutive elements (agentlenshq.com, "Transformers
+4.40 performance upgrades for OpenAI GPT-OSS ...", section "What MXFP4 Is").
+Packed layout: codes uint8 [rows, cols/2] (even element in the low nibble),
+scales uint8 [rows, cols/32].
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (Mxfp4Error, Mxfp4LibraryMissing, SCALE_CEIL, SCALE_FLOOR, W4A4, W4A16)
+
+__all__ = [
+    "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_gemm_workspace_size",
+    "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
+    "moe_mxfp4_workspace_size", "mxfp4_get_device_status", "Mxfp4Error", "Mxfp4LibraryMissing",
+    "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
+]
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _p(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _empty(shape, dtype, like):
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+def mxfp4_quantize(x: torch.Tensor, rule: int = SCALE_FLOOR, codes=None, scales=None, stream=None):
+    """x bf16/fp32 [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [rows, cols/32])."""
+    lib = _lib.load()
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    R, C = x.shape
+    dt = {torch.bfloat16: _lib.IN_BF16, torch.float32: _lib.IN_F32}.get(x.dtype)
+    if dt is None:
+        raise ValueError("x must be bf16 or fp32")
+    codes = _empty((R, C // 2), torch.uint8, x) if codes is None else codes
+    scales = _empty((R, C // 32), torch.uint8, x) if scales is None else scales
+    _lib.check("mxfp4_quantize", lib.mxfp4_quantize(_p(x), dt, R, C, _p(codes), _p(scales),
+                                                    int(rule), _stream(stream)))
+    return codes, scales
+
+
+def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, out=None, stream=None):
+    """codes uint8 [rows, cols/2] + scales uint8 [rows, cols/32] -> bf16 [rows, cols]."""
+    lib = _lib.load()
+    R, half = codes.shape
+    C = 2 * half
+    out = _empty((R, C), torch.bfloat16, codes) if out is None else out
+    _lib.check("mxfp4_dequantize", lib.mxfp4_dequantize(_p(codes), _p(scales), R, C, _p(out),
+                                                        _stream(stream)))
+    return out
+
+
+def mxfp4_gemm_workspace_size(M, K, N, mode=W4A16) -> int:
+    return int(_lib.load().mxfp4_gemm_workspace_size(M, K, N, int(mode)))
+
+
+def mxfp4_gemm(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, mode: int = W4A16,
+               out=None, ws=None, stream=None):
+    """y bf16 [M, N] = x bf16 [M, K] . dequant(W)^T, W codes [N, K/2] + scales [N, K/32]."""
+    lib = _lib.load()
+    M, K = x.shape
+    N = w_codes.shape[0]
+    out = _empty((M, N), torch.bfloat16, x) if out is None else out
+    need = mxfp4_gemm_workspace_size(M, K, N, mode)
+    if ws is None and need:
+        ws = _empty((need,), torch.uint8, x)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _lib.check("mxfp4_gemm", lib.mxfp4_gemm(_p(x), M, K, _p(w_codes), _p(w_scales), N, _p(out),
+                                            int(mode), _p(ws), nbytes, _stream(stream)))
+    return out
+
+
+def moe_mxfp4_route_workspace_size(T, E, top_k) -> int:
+    return int(_lib.load().moe_mxfp4_route_workspace_size(T, E, top_k))
+
+
+def moe_mxfp4_route(logits: torch.Tensor, top_k: int, ws=None, stream=None):
+    """Top-k routing + expert-sorted permutation; returns a dict of device tensors
+    ids [T, k] i32, weights [T, k] f32, counts [E] i32, offsets [E+1] i32,
+    perm [T*k] i32, inv [T*k] i32."""
+    lib = _lib.load()
+    T, E = logits.shape
+    P = T * top_k
+    out = dict(ids=_empty((T, top_k), torch.int32, logits),
+               weights=_empty((T, top_k), torch.float32, logits),
+               counts=_empty((E,), torch.int32, logits),
+               offsets=_empty((E + 1,), torch.int32, logits),
+               perm=_empty((P,), torch.int32, logits),
+               inv=_empty((P,), torch.int32, logits))
+    need = moe_mxfp4_route_workspace_size(T, E, top_k)
+    ws = _empty((need,), torch.uint8, logits) if ws is None else ws
+    _lib.check("moe_mxfp4_route", lib.moe_mxfp4_route(
+        _p(logits), T, E, top_k, _p(out["ids"]), _p(out["weights"]), _p(out["counts"]),
+        _p(out["offsets"]), _p(out["perm"]), _p(out["inv"]), _p(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def moe_mxfp4_workspace_size(T, H, I, E, top_k, mode=W4A16) -> int:
+    return int(_lib.load().moe_mxfp4_workspace_size(T, H, I, E, top_k, int(mode)))
+
+
+def moe_mxfp4_mlp(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13_codes, w13_scales,
+                  w2_codes, w2_scales, mode: int = W4A16, out=None, ws=None, stream=None):
+    """One MoE expert-MLP layer with MXFP4 expert weights (see include/mxfp4.h).
+    x bf16 [T, H]; logits f32 [T, E]; w13 codes [E, 2I, H/2] + scales [E, 2I, H/32];
+    w2 codes [E, H, I/2] + scales [E, H, I/32] -> out bf16 [T, H]."""
+    lib = _lib.load()
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w13_codes.shape[1] // 2
+    out = _empty((T, H), torch.bfloat16, x) if out is None else out
+    need = moe_mxfp4_workspace_size(T, H, I, E, top_k, mode)
+    ws = _empty((need,), torch.uint8, x) if ws is None else ws
+    _lib.check("moe_mxfp4_mlp", lib.moe_mxfp4_mlp(
+        _p(x), T, H, _p(logits), E, top_k, _p(w13_codes), _p(w13_scales), I, _p(w2_codes),
+        _p(w2_scales), _p(out), int(mode), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return out
+
+
+def mxfp4_get_device_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status word."""
+    return int(_lib.load().mxfp4_get_device_status(_stream(stream)))

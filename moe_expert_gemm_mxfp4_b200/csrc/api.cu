@@ -1,0 +1,417 @@
+// C ABI of the library (declared in include/mxfp4.h): argument validation,
+// workspace carving, TMA tensor-map encoding and the launch sequence of each
+// entry point.  No allocation, no host synchronization (except in
+// mxfp4_get_device_status), no printing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+
+// Per-device status word written by kernels whose waits ran out of time.
+__device__ unsigned g_mxfp4_status;
+
+namespace {
+
+thread_local int tl_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0, minor = 0;
+    unsigned* status = nullptr;
+    bool ready = false;
+};
+
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+mxfp4_status cuda_fail(cudaError_t e) {
+    tl_last_cuda_error = static_cast<int>(e);
+    return MXFP4_ERR_CUDA;
+}
+
+// Device properties and the status word's address, once per device.
+mxfp4_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return MXFP4_ERR_ARCH;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if (d.major == 10 && d.minor == 0) {
+            void* p = nullptr;
+            if ((e = cudaGetSymbolAddress(&p, g_mxfp4_status)) != cudaSuccess) return cuda_fail(e);
+            d.status = static_cast<unsigned*>(p);
+        }
+        d.ready = true;
+    }
+    if (!(d.major == 10 && d.minor == 0)) return MXFP4_ERR_ARCH;
+    *out = &d;
+    return MXFP4_OK;
+}
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Packed codes of G groups as a 3-D tensor {K/2 bytes, rows, G}; box {32, box_rows, 1};
+// 32-byte swizzle (conflict-free 16-B reads of one row per thread).
+mxfp4_status encode_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t K, int64_t rows,
+                              int64_t G, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(G)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2),
+                                   static_cast<cuuint64_t>(rows * (K / 2))};
+    const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(codes), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
+}
+
+// bf16 activations {K, rows}; box {64, nt}; 128-byte swizzle (UMMA K-major SW128 layout).
+mxfp4_status encode_act_map(CUtensorMap* m, const void* x, int64_t K, int64_t rows, int nt) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(nt)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace of moe_mxfp4_mlp, carved in this order (256-byte aligned pieces).
+struct MoeWs {
+    int32_t* ids;
+    float* weights;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm;
+    int32_t* inv;
+    float* w_sorted;
+    void* route_tmp;
+    void* x_sorted;   // bf16 [P, H]
+    void* h;          // bf16 [P, I]
+    void* y_sorted;   // bf16 [P, H]; W4A4 also parks the quantized x [T, H] here first
+    size_t bytes;
+};
+
+MoeWs carve_moe(void* base, int64_t T, int64_t H, int64_t I, int64_t E, int top_k) {
+    const int64_t P = T * top_k;
+    MoeWs w{};
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        void* p = base ? static_cast<uint8_t*>(base) + off : nullptr;
+        off = align_up(off + n, 256);
+        return p;
+    };
+    w.ids = static_cast<int32_t*>(take(P * 4));
+    w.weights = static_cast<float*>(take(P * 4));
+    w.counts = static_cast<int32_t*>(take(E * 4));
+    w.offsets = static_cast<int32_t*>(take((E + 1) * 4));
+    w.perm = static_cast<int32_t*>(take(P * 4));
+    w.inv = static_cast<int32_t*>(take(P * 4));
+    w.w_sorted = static_cast<float*>(take(P * 4));
+    w.route_tmp = take(mx::route_tmp_bytes(T, E, top_k));
+    w.x_sorted = take(static_cast<size_t>(P) * H * 2);
+    w.h = take(static_cast<size_t>(P) * I * 2);
+    w.y_sorted = take(static_cast<size_t>(P) * H * 2);
+    w.bytes = off;
+    return w;
+}
+
+int gemm_grid(const DeviceInfo* d, int64_t tile_bound) {
+    int64_t g = tile_bound < d->sm_count ? tile_bound : d->sm_count;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mxfp4_status_string(mxfp4_status s) {
+    switch (s) {
+        case MXFP4_OK: return "MXFP4_OK";
+        case MXFP4_ERR_INVALID_ARG: return "MXFP4_ERR_INVALID_ARG";
+        case MXFP4_ERR_UNSUPPORTED_SHAPE: return "MXFP4_ERR_UNSUPPORTED_SHAPE";
+        case MXFP4_ERR_MISALIGNED: return "MXFP4_ERR_MISALIGNED";
+        case MXFP4_ERR_ARCH: return "MXFP4_ERR_ARCH";
+        case MXFP4_ERR_WORKSPACE: return "MXFP4_ERR_WORKSPACE";
+        case MXFP4_ERR_CUDA: return "MXFP4_ERR_CUDA";
+        case MXFP4_ERR_TIMEOUT: return "MXFP4_ERR_TIMEOUT";
+    }
+    return "MXFP4_ERR_UNKNOWN";
+}
+
+int mxfp4_last_cuda_error(void) { return tl_last_cuda_error; }
+
+mxfp4_status mxfp4_get_device_status(void* stream) {
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned v = 0;
+    if ((e = cudaMemcpyFromSymbolAsync(&v, g_mxfp4_status, sizeof v, 0, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+        return cuda_fail(e);
+    const unsigned zero = 0;
+    if ((e = cudaMemcpyToSymbolAsync(g_mxfp4_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+        return cuda_fail(e);
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e);
+    return static_cast<mxfp4_status>(v);
+}
+
+mxfp4_status mxfp4_quantize(const void* x, mxfp4_in_dtype dt, int64_t rows, int64_t cols,
+                            uint8_t* codes, uint8_t* scales, mxfp4_scale_rule rule, void* stream) {
+    if (!x || !codes || !scales) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (dt != MXFP4_IN_BF16 && dt != MXFP4_IN_F32) return MXFP4_ERR_INVALID_ARG;
+    if (rule != MXFP4_SCALE_FLOOR && rule != MXFP4_SCALE_CEIL) return MXFP4_ERR_INVALID_ARG;
+    if (cols % 32 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t{1} << 40) / cols) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaError_t e = mx::launch_quantize(x, dt == MXFP4_IN_F32, rows, cols, codes, scales,
+                                        static_cast<int>(rule), d->sm_count,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                              int64_t cols, void* out_bf16, void* stream) {
+    if (!codes || !scales || !out_bf16) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (cols % 32 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows > (int64_t{1} << 40) / cols) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(out_bf16)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaError_t e = mx::launch_dequantize(codes, scales, rows, cols, out_bf16, d->sm_count,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp4_mode mode) {
+    (void)N;
+    if (mode != MXFP4_W4A4 || M <= 0 || K <= 0) return 0;
+    return align_up(static_cast<size_t>(M) * K * 2, 256);
+}
+
+mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t* w_codes,
+                        const uint8_t* w_scales, int64_t N, void* y_bf16, mxfp4_mode mode,
+                        void* ws, size_t ws_bytes, void* stream) {
+    if (!x_bf16 || !w_codes || !w_scales || !y_bf16) return MXFP4_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0 || N <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) || K >= (int64_t{1} << 24))
+        return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y_bf16))
+        return MXFP4_ERR_MISALIGNED;
+    const size_t need = mxfp4_gemm_workspace_size(M, K, N, mode);
+    if (need > 0 && (!ws || ws_bytes < need)) return MXFP4_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const void* xa = x_bf16;
+    if (mode == MXFP4_W4A4) {
+        cudaError_t e = mx::launch_qdq_bf16(x_bf16, M, K, ws, d->sm_count, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        xa = ws;
+    }
+    const int nt = mx::pick_token_tile(M, 1);
+    CUtensorMap tw, tx;
+    if ((st = encode_codes_map(&tw, w_codes, K, N, 1, 128)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, xa, K, M, nt)) != MXFP4_OK) return st;
+    mx::GemmArgs a{};
+    a.w_scales = w_scales;
+    a.offsets = nullptr;
+    a.m_single = static_cast<int>(M);
+    a.G = 1;
+    a.K = static_cast<int>(K);
+    a.rows_w = static_cast<int>(N);
+    a.I = 0;
+    a.n_ftiles = static_cast<int>((N + 127) / 128);
+    a.out = y_bf16;
+    a.out_ld = N;
+    a.n_valid_feat = static_cast<int>(N);
+    a.row_w = nullptr;
+    a.status = d->status;
+    const int64_t tiles = ((M + nt - 1) / nt) * a.n_ftiles;
+    cudaError_t e = mx::launch_grouped_gemm(mx::EPI_PLAIN, nt, tw, tx, a, gemm_grid(d, tiles), s);
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+static mxfp4_status check_route_args(const float* logits, int64_t T, int64_t E, int32_t top_k) {
+    if (!logits) return MXFP4_ERR_INVALID_ARG;
+    if (T <= 0 || E <= 0 || top_k <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (E > 256 || top_k > 8 || top_k > E) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (T * top_k >= (int64_t{1} << 31)) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    return MXFP4_OK;
+}
+
+size_t moe_mxfp4_route_workspace_size(int64_t T, int64_t E, int32_t top_k) {
+    if (T <= 0 || E <= 0 || top_k <= 0) return 0;
+    return align_up(mx::route_tmp_bytes(T, E, top_k), 256);
+}
+
+mxfp4_status moe_mxfp4_route(const float* router_logits, int64_t T, int64_t E, int32_t top_k,
+                             int32_t* ids, float* weights, int32_t* counts, int32_t* offsets,
+                             int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+    mxfp4_status st = check_route_args(router_logits, T, E, top_k);
+    if (st != MXFP4_OK) return st;
+    if (!ids || !weights || !counts || !offsets || !perm || !inv) return MXFP4_ERR_INVALID_ARG;
+    if (!aligned16(router_logits) || !aligned16(ids) || !aligned16(weights) || !aligned16(counts) ||
+        !aligned16(offsets) || !aligned16(perm) || !aligned16(inv))
+        return MXFP4_ERR_MISALIGNED;
+    const size_t need = moe_mxfp4_route_workspace_size(T, E, top_k);
+    if (!ws || ws_bytes < need) return MXFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((st = device_info(&d)) != MXFP4_OK) return st;
+    cudaError_t e = mx::launch_route(router_logits, T, E, top_k, ids, weights, counts, offsets, perm,
+                                     inv, nullptr, ws, nullptr, 0, nullptr, d->sm_count,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k,
+                                mxfp4_mode mode) {
+    (void)mode;
+    if (T <= 0 || H <= 0 || I <= 0 || E <= 0 || top_k <= 0) return 0;
+    return carve_moe(nullptr, T, H, I, E, top_k).bytes;
+}
+
+mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float* router_logits,
+                           int64_t E, int32_t top_k, const uint8_t* w13_codes,
+                           const uint8_t* w13_scales, int64_t I, const uint8_t* w2_codes,
+                           const uint8_t* w2_scales, void* out_bf16, mxfp4_mode mode, void* ws,
+                           size_t ws_bytes, void* stream) {
+    mxfp4_status st = check_route_args(router_logits, T, E, top_k);
+    if (st != MXFP4_OK) return st;
+    if (!x_bf16 || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !out_bf16)
+        return MXFP4_ERR_INVALID_ARG;
+    if (H <= 0 || I <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
+    if (H % 64 != 0 || I % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (H >= (int64_t{1} << 24) || I >= (int64_t{1} << 24)) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(router_logits) || !aligned16(w13_codes) ||
+        !aligned16(w13_scales) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
+        !aligned16(out_bf16))
+        return MXFP4_ERR_MISALIGNED;
+    const size_t need = moe_mxfp4_workspace_size(T, H, I, E, top_k, mode);
+    if (!ws || ws_bytes < need) return MXFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((st = device_info(&d)) != MXFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const MoeWs w = carve_moe(ws, T, H, I, E, top_k);
+    const int64_t P = T * top_k;
+    cudaError_t e;
+
+    const void* x_src = x_bf16;
+    if (mode == MXFP4_W4A4) {   // activations on the MXFP4 grid, rows along H
+        if ((e = mx::launch_qdq_bf16(x_bf16, T, H, w.y_sorted, d->sm_count, s)) != cudaSuccess)
+            return cuda_fail(e);
+        x_src = w.y_sorted;
+    }
+    if ((e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets,
+                              w.perm, w.inv, w.w_sorted, w.route_tmp, x_src, H, w.x_sorted,
+                              d->sm_count, s)) != cudaSuccess)
+        return cuda_fail(e);
+
+    const int nt = mx::pick_token_tile(P, E);
+    const int64_t tok_tiles = (P + nt - 1) / nt + E;
+
+    // gate/up projection with the SwiGLU epilogue -> h [P, I]
+    CUtensorMap tw, tx;
+    if ((st = encode_codes_map(&tw, w13_codes, H, 2 * I, E, 64)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, w.x_sorted, H, P, nt)) != MXFP4_OK) return st;
+    mx::GemmArgs a{};
+    a.w_scales = w13_scales;
+    a.offsets = w.offsets;
+    a.m_single = 0;
+    a.G = static_cast<int>(E);
+    a.K = static_cast<int>(H);
+    a.rows_w = static_cast<int>(2 * I);
+    a.I = static_cast<int>(I);
+    a.n_ftiles = static_cast<int>(I / 64);
+    a.out = w.h;
+    a.out_ld = I;
+    a.n_valid_feat = static_cast<int>(I);
+    a.row_w = nullptr;
+    a.status = d->status;
+    if ((e = mx::launch_grouped_gemm(mx::EPI_SWIGLU, nt, tw, tx, a,
+                                     gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
+        return cuda_fail(e);
+
+    if (mode == MXFP4_W4A4) {   // h on the MXFP4 grid, rows along I (in place)
+        if ((e = mx::launch_qdq_bf16(w.h, P, I, w.h, d->sm_count, s)) != cudaSuccess)
+            return cuda_fail(e);
+    }
+
+    // down projection, routing weight applied in fp32 -> y_sorted [P, H]
+    if ((st = encode_codes_map(&tw, w2_codes, I, H, E, 128)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, w.h, I, P, nt)) != MXFP4_OK) return st;
+    a.w_scales = w2_scales;
+    a.K = static_cast<int>(I);
+    a.rows_w = static_cast<int>(H);
+    a.I = 0;
+    a.n_ftiles = static_cast<int>((H + 127) / 128);
+    a.out = w.y_sorted;
+    a.out_ld = H;
+    a.n_valid_feat = static_cast<int>(H);
+    a.row_w = w.w_sorted;
+    if ((e = mx::launch_grouped_gemm(mx::EPI_WEIGHTED, nt, tw, tx, a,
+                                     gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
+        return cuda_fail(e);
+
+    // deterministic combine in slot order
+    if ((e = mx::launch_combine(w.y_sorted, w.inv, T, top_k, H, out_bf16, d->sm_count, s)) !=
+        cudaSuccess)
+        return cuda_fail(e);
+    return MXFP4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// Internal (non-exported) interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mx {
+
+enum EpiMode { EPI_PLAIN = 0, EPI_SWIGLU = 1, EPI_WEIGHTED = 2 };
+
+// Arguments of the grouped W4A16 GEMM (see gemm.cu).
+struct GemmArgs {
+    const uint8_t* w_scales;   // [G, rows_w, K/32]
+    const int32_t* offsets;    // [G+1] row offsets of each group, or nullptr (one group)
+    int m_single;              // rows of the single group when offsets == nullptr
+    int G;
+    int K;
+    int rows_w;                // weight rows per group
+    int I;                     // SWIGLU: gate rows [0, I), up rows [I, 2I)
+    int n_ftiles;              // feature tiles per group
+    void* out;                 // bf16 output, row-major
+    int64_t out_ld;            // elements per output row
+    int n_valid_feat;          // valid output columns
+    const float* row_w;        // WEIGHTED: per-row scalar
+    unsigned* status;          // device status word
+};
+
+cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t cols,
+                            uint8_t* codes, uint8_t* scales, int rule, int sm_count,
+                            cudaStream_t stream);
+cudaError_t launch_qdq_bf16(const void* x, int64_t rows, int64_t cols, void* out, int sm_count,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                              int64_t cols, void* out, int sm_count, cudaStream_t stream);
+size_t route_tmp_bytes(int64_t T, int64_t E, int top_k);
+cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, int32_t* ids,
+                         float* weights, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* inv, float* w_sorted, void* tmp, const void* x, int64_t H,
+                         void* x_sorted, int sm_count, cudaStream_t stream);
+cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, int top_k,
+                           int64_t H, void* out, int sm_count, cudaStream_t stream);
+int pick_token_tile(int64_t rows, int64_t groups);
+cudaError_t launch_grouped_gemm(int mode, int nt, const CUtensorMap& tmap_w,
+                                const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
+                                cudaStream_t stream);
+
+}  // namespace mx

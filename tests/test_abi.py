@@ -1,0 +1,89 @@
+"""The C ABI library builds for sm_100a, loads, exports every function the public
+header declares, and rejects invalid arguments on the host before touching the
+GPU (these checks run without a GPU: they fail before any CUDA call)."""
+import ctypes
+
+import pytest
+
+import moe_expert_gemm_mxfp4_b200 as mx
+from moe_expert_gemm_mxfp4_b200 import _lib
+from moe_expert_gemm_mxfp4_b200 import build as mxbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mxbuild.build()
+    return _lib.load()
+
+
+def test_header_declares_the_api():
+    names = _lib.header_symbols()
+    for n in ("mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "moe_mxfp4_mlp",
+              "moe_mxfp4_route", "mxfp4_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_header_symbol(lib):
+    for name in _lib.header_symbols():
+        assert hasattr(lib, name), f"{name} declared in include/mxfp4.h but not exported"
+        assert name in _lib._SIGS, f"{name} has no ctypes signature in the binding"
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.mxfp4_status_string(code).startswith(b"MXFP4_")
+
+
+A = ctypes.c_void_p(0x10000)      # aligned fake device pointer (never dereferenced)
+U = ctypes.c_void_p(0x10001)      # misaligned fake pointer
+N = ctypes.c_void_p(0)
+
+
+def test_quantize_argument_checks(lib):
+    q = lib.mxfp4_quantize
+    assert q(N, 0, 4, 64, A, A, 0, N) == _lib.ERR_INVALID_ARG
+    assert q(A, 0, 0, 64, A, A, 0, N) == _lib.ERR_INVALID_ARG
+    assert q(A, 0, 4, -32, A, A, 0, N) == _lib.ERR_INVALID_ARG
+    assert q(A, 7, 4, 64, A, A, 0, N) == _lib.ERR_INVALID_ARG
+    assert q(A, 0, 4, 64, A, A, 9, N) == _lib.ERR_INVALID_ARG
+    assert q(A, 0, 4, 48, A, A, 0, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert q(U, 0, 4, 64, A, A, 0, N) == _lib.ERR_MISALIGNED
+    assert lib.mxfp4_dequantize(A, N, 4, 64, A, N) == _lib.ERR_INVALID_ARG
+    assert lib.mxfp4_dequantize(A, A, 4, 40, A, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert lib.mxfp4_dequantize(A, A, 4, 64, U, N) == _lib.ERR_MISALIGNED
+
+
+def test_gemm_argument_checks(lib):
+    g = lib.mxfp4_gemm
+    assert g(A, 8, 256, A, A, 512, N, 0, N, 0, N) == _lib.ERR_INVALID_ARG
+    assert g(A, 0, 256, A, A, 512, A, 0, N, 0, N) == _lib.ERR_INVALID_ARG
+    assert g(A, 8, 256, A, A, 512, A, 5, N, 0, N) == _lib.ERR_INVALID_ARG
+    assert g(A, 8, 96, A, A, 512, A, 0, N, 0, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert g(A, 8, 256, U, A, 512, A, 0, N, 0, N) == _lib.ERR_MISALIGNED
+    assert g(A, 8, 256, A, A, 512, A, 1, N, 0, N) == _lib.ERR_WORKSPACE   # W4A4 needs ws
+    assert lib.mxfp4_gemm_workspace_size(8, 256, 512, 0) == 0
+    assert lib.mxfp4_gemm_workspace_size(8, 256, 512, 1) >= 8 * 256 * 2
+
+
+def test_route_and_moe_argument_checks(lib):
+    r = lib.moe_mxfp4_route
+    assert r(A, 64, 32, 0, A, A, A, A, A, A, A, 1 << 20, N) == _lib.ERR_INVALID_ARG
+    assert r(A, 64, 32, 9, A, A, A, A, A, A, A, 1 << 20, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert r(A, 64, 300, 4, A, A, A, A, A, A, A, 1 << 20, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert r(A, 64, 3, 4, A, A, A, A, A, A, A, 1 << 20, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert r(A, 64, 32, 4, A, A, A, A, A, A, N, 0, N) == _lib.ERR_WORKSPACE
+    m = lib.moe_mxfp4_mlp
+    big = 1 << 40
+    assert m(A, 64, 2880, A, 32, 4, A, A, 2880, A, A, A, 0, N, 0, N) == _lib.ERR_WORKSPACE
+    assert m(A, 64, 2880 + 32, A, 32, 4, A, A, 2880, A, A, A, 0, A, big, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert m(A, 64, 2880, A, 32, 4, A, A, 2880 + 32, A, A, A, 0, A, big, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert m(A, 64, 2880, A, 32, 4, U, A, 2880, A, A, A, 0, A, big, N) == _lib.ERR_MISALIGNED
+    assert m(A, 64, 2880, A, 32, 4, A, A, 2880, A, A, A, 3, A, big, N) == _lib.ERR_INVALID_ARG
+    ws = lib.moe_mxfp4_workspace_size(64, 2880, 2880, 32, 4, 0)
+    assert ws >= 64 * 4 * (2880 * 2 * 2 + 2880 * 2)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(_lib, "_LIB", None)
+    with pytest.raises(_lib.Mxfp4LibraryMissing):
+        _lib.load(str(tmp_path / "nope.so"))

@@ -1,0 +1,106 @@
+"""GPU parity of moe_mxfp4_mlp (the whole MoE expert-MLP layer) against the fp64
+oracle: every token for small layers and the decode workload, a seeded sample of
+tokens (computed one by one by the oracle) for the prefill and 120b-shaped
+workloads at full size, in the launch configuration the benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import moe_expert_gemm_mxfp4_b200 as mx
+from moe_expert_gemm_mxfp4_b200 import inputs
+from helpers import assert_close_tol, bits_of, f64_of, oracle_quantize_weights
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+class Layer:
+    """MoE layer inputs: fp32 weights quantized by the oracle, kept on host and device."""
+
+    def __init__(self, cfg, T=None):
+        self.cfg = cfg
+        self.x, self.logits = inputs.moe_activations(cfg, T)
+        E, I, H = cfg.E, cfg.I, cfg.H
+        self.w13c = np.empty((E, 2 * I, H // 2), np.uint8)
+        self.w13s = np.empty((E, 2 * I, H // 32), np.uint8)
+        self.w2c = np.empty((E, H, I // 2), np.uint8)
+        self.w2s = np.empty((E, H, I // 32), np.uint8)
+        for e in range(E):
+            w13, w2 = inputs.expert_weights(cfg, e)
+            self.w13c[e], self.w13s[e] = oracle_quantize_weights(w13)
+            self.w2c[e], self.w2s[e] = oracle_quantize_weights(w2)
+        self.dev = [torch.from_numpy(a).to(DEV) for a in (self.w13c, self.w13s, self.w2c, self.w2s)]
+
+    def gpu(self, mode=mx.W4A16):
+        out = mx.moe_mxfp4_mlp(self.x.to(DEV), self.logits.to(DEV), self.cfg.top_k, *self.dev, mode=mode)
+        torch.cuda.synchronize()
+        assert mx.mxfp4_get_device_status() == 0
+        return f64_of(out)
+
+    def ref(self, mode="w4a16", tokens=None):
+        return oracle.moe_mlp(bits_of(self.x), self.logits.numpy(), self.cfg.top_k, self.w13c,
+                              self.w13s, self.w2c, self.w2s, mode=mode, tokens=tokens)
+
+
+def _small(T, H, I, E, k, seed, hot=()):
+    return inputs.MoEConfig("small", seed=seed, T=T, E=E, top_k=k, H=H, I=I,
+                            hot_experts=hot, hot_bias=2.0 if hot else 0.0, w_std=0.05)
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [(1, 64, 64, 1, 1), (5, 128, 64, 4, 2), (37, 192, 128, 8, 2),
+                                       (64, 256, 320, 16, 4), (300, 128, 192, 5, 3),
+                                       (513, 64, 128, 3, 1)])
+def test_moe_small_all_tokens(T, H, I, E, k):
+    L = Layer(_small(T, H, I, E, k, seed=T + H + I + E + k))
+    assert_close_tol(L.gpu(), L.ref(), what=f"moe T={T} H={H} I={I} E={E} k={k}")
+
+
+def test_moe_small_imbalanced_and_empty_experts():
+    L = Layer(_small(200, 128, 128, 12, 2, seed=99, hot=(0, 1)))
+    assert_close_tol(L.gpu(), L.ref(), what="imbalanced")
+
+
+@pytest.fixture(scope="module")
+def decode_layer():
+    return Layer(inputs.MOE_CONFIGS["moe_decode"])
+
+
+def test_moe_decode_workload_all_tokens(decode_layer):
+    L = decode_layer
+    assert_close_tol(L.gpu(), L.ref(), what="decode T=64 E=32")
+
+
+def _sample(T, n, seed):
+    g = torch.Generator().manual_seed(seed)
+    return np.sort(torch.randperm(T, generator=g)[:n].numpy())
+
+
+def test_moe_prefill_workload_sampled():
+    L = Layer(inputs.MOE_CONFIGS["moe_prefill"])
+    out = L.gpu()
+    tok = _sample(L.cfg.T, 96, 1)
+    assert_close_tol(out[tok], L.ref(tokens=tok), what="prefill T=8192 (sampled)")
+    assert np.all(np.isfinite(out))
+
+
+@pytest.fixture(scope="module")
+def l120():
+    return Layer(inputs.MOE_CONFIGS["moe_120b"])
+
+
+def test_moe_120b_w4a16_sampled(l120):
+    out = l120.gpu(mx.W4A16)
+    tok = _sample(l120.cfg.T, 64, 2)
+    assert_close_tol(out[tok], l120.ref(tokens=tok), what="120b W4A16 (sampled)")
+
+
+def test_moe_120b_w4a4_sampled(l120):
+    out = l120.gpu(mx.W4A4)
+    tok = _sample(l120.cfg.T, 64, 3)
+    assert_close_tol(out[tok], l120.ref(mode="w4a4", tokens=tok), what="120b W4A4 (sampled)")
+
+
+def test_moe_small_w4a4_all_tokens():
+    L = Layer(_small(64, 256, 192, 8, 2, seed=5))
+    assert_close_tol(L.gpu(mx.W4A4), L.ref(mode="w4a4"), what="small W4A4")
