@@ -127,7 +127,7 @@ struct MoeWs {
     void* route_tmp;
     void* x_sorted;   // bf16 [P, H]
     void* h;          // bf16 [P, I]
-    void* y_sorted;   // bf16 [P, H]; W4A4 also parks the quantized x [T, H] here first
+    void* y_sorted;   // fp32 [P, H]; W4A4 also parks the quantized x (bf16 [T, H]) here first
     size_t bytes;
 };
 
@@ -150,7 +150,7 @@ MoeWs carve_moe(void* base, int64_t T, int64_t H, int64_t I, int64_t E, int top_
     w.route_tmp = take(mx::route_tmp_bytes(T, E, top_k));
     w.x_sorted = take(static_cast<size_t>(P) * H * 2);
     w.h = take(static_cast<size_t>(P) * I * 2);
-    w.y_sorted = take(static_cast<size_t>(P) * H * 2);
+    w.y_sorted = take(static_cast<size_t>(P) * H * 4);
     w.bytes = off;
     return w;
 }
@@ -391,7 +391,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
             return cuda_fail(e);
     }
 
-    // down projection, routing weight applied in fp32 -> y_sorted [P, H]
+    // down projection, routing weight applied in fp32 -> y_sorted fp32 [P, H]
     if ((st = encode_codes_map(&tw, w2_codes, I, H, E, 128)) != MXFP4_OK) return st;
     if ((st = encode_act_map(&tx, w.h, I, P, nt)) != MXFP4_OK) return st;
     a.w_scales = w2_scales;

@@ -6,7 +6,7 @@
 // with fp32 accumulation, and applies one of three fused epilogues:
 //   PLAIN     y = bf16(D)
 //   SWIGLU    h = bf16(SiLU(D_gate) * D_up), W rows [0, I) gate and [I, 2I) up
-//   WEIGHTED  y = bf16(w_row * D), w_row = the routing weight of the row
+//   WEIGHTED  y = w_row * D (fp32 out), w_row = the routing weight of the row
 // (the gpt-oss expert MLP run on MXFP4 weights; agentlenshq.com, "Transformers
 // 4.40 performance upgrades for OpenAI GPT-OSS ...", sections "What MXFP4 Is"
 // and "Zero-Build Kernels from the Hub").
@@ -387,9 +387,12 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         for (int n = 0; n < 16; ++n) {
                             const int tok = 16 * c + n;
                             if (tok < ti.mrows) {
-                                float val = __uint_as_float(v[n]);
-                                if (MODE == EPI_WEIGHTED) val *= args.row_w[ti.row0 + tok];
-                                store_bf16(args.out, static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat, val);
+                                const int64_t idx = static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat;
+                                const float val = __uint_as_float(v[n]);
+                                if (MODE == EPI_WEIGHTED)   // fp32 out: one rounding, in the combine
+                                    reinterpret_cast<float*>(args.out)[idx] = val * args.row_w[ti.row0 + tok];
+                                else
+                                    store_bf16(args.out, idx, val);
                             }
                         }
                     }

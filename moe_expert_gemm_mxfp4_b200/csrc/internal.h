@@ -20,7 +20,7 @@ struct GemmArgs {
     int rows_w;                // weight rows per group
     int I;                     // SWIGLU: gate rows [0, I), up rows [I, 2I)
     int n_ftiles;              // feature tiles per group
-    void* out;                 // bf16 output, row-major
+    void* out;                 // output, row-major: bf16 (PLAIN, SWIGLU) or fp32 (WEIGHTED)
     int64_t out_ld;            // elements per output row
     int n_valid_feat;          // valid output columns
     const float* row_w;        // WEIGHTED: per-row scalar

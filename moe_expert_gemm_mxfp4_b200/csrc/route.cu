@@ -17,7 +17,7 @@
 //                     offsets (exclusive scan over experts);
 //   route_scatter     position of every pair, perm / inv / sorted weights, and
 //                     optionally the gather of its token row;
-//   moe_combine       out[t] = sum_j y[inv[t*k + j]] in slot order (fp32).
+//   moe_combine       out[t] = bf16(sum_j y[inv[t*k + j]]), fp32 rows summed in slot order.
 #include "common.cuh"
 #include "internal.h"
 
@@ -198,41 +198,36 @@ route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
     }
 }
 
-__device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t w) {
-    a += __uint_as_float(w << 16);
-    b += __uint_as_float(w & 0xFFFF0000u);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// One warp per token; the k rows are summed in slot order j = 0..k-1 in fp32.
+// One warp per token; its k fp32 rows are summed in slot order j = 0..k-1 and
+// rounded once to bf16.
 __global__ void __launch_bounds__(kRouteThreads)
-moe_combine_kernel(const uint4* __restrict__ y_sorted, const int32_t* __restrict__ inv,
-                   int64_t T, int k, int64_t row_vec, uint4* __restrict__ out) {
+moe_combine_kernel(const float4* __restrict__ y_sorted, const int32_t* __restrict__ inv,
+                   int64_t T, int k, int64_t row_vec8, uint4* __restrict__ out) {
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t t = warp0; t < T; t += nwarps) {
         int64_t rows[kMaxTopK];
         for (int j = 0; j < k; ++j) rows[j] = inv[t * k + j];
-        for (int64_t c = lane; c < row_vec; c += 32) {
+        for (int64_t c = lane; c < row_vec8; c += 32) {
             float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < k; ++j) {
-                const uint4 v = __ldcs(y_sorted + rows[j] * row_vec + c);
-                add_bf16x2(a[0], a[1], v.x);
-                add_bf16x2(a[2], a[3], v.y);
-                add_bf16x2(a[4], a[5], v.z);
-                add_bf16x2(a[6], a[7], v.w);
+                const float4* src = y_sorted + (rows[j] * row_vec8 + c) * 2;
+                const float4 u = __ldcs(src), v = __ldcs(src + 1);
+                a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
+                a[4] += v.x; a[5] += v.y; a[6] += v.z; a[7] += v.w;
             }
             uint4 o;
             o.x = pack_bf16x2(a[0], a[1]);
             o.y = pack_bf16x2(a[2], a[3]);
             o.z = pack_bf16x2(a[4], a[5]);
             o.w = pack_bf16x2(a[6], a[7]);
-            out[t * row_vec + c] = o;
+            out[t * row_vec8 + c] = o;
         }
     }
 }
@@ -273,7 +268,7 @@ cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, 
     const int64_t cap = static_cast<int64_t>(sm_count) * 8;
     if (grid > cap) grid = cap;
     moe_combine_kernel<<<static_cast<unsigned>(grid), kRouteThreads, 0, stream>>>(
-        static_cast<const uint4*>(y_sorted), inv, T, top_k, H / 8, static_cast<uint4*>(out));
+        static_cast<const float4*>(y_sorted), inv, T, top_k, H / 8, static_cast<uint4*>(out));
     return cudaGetLastError();
 }
 
