@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP4 MoE expert-MLP layer on B200 (one JSON line on stdout).
+
+A step is one forward of the gpt-oss-20b-shaped MoE layer on the prefill
+workload (T = 8192 tokens, H = I = 2880, 32 experts, top-4, MXFP4 expert
+weights, W4A16): routing + gather, grouped gate/up GEMM with the SwiGLU
+epilogue, grouped down GEMM with the routing weight, combine.  `value` is the
+layer's algorithmic TFLOP/s, 2 * T * k * (2I*H + H*I) flops per step, with all
+inputs resident in HBM.  The same JSON line also carries, measured in the same
+run: quantize / dequantize GB/s on the bf16 [4096, 11520] tensor, the decode
+layer (T = 64) as expert-weight GB/s, and the 120b-shaped layer (T = 4096,
+128 experts) in W4A16 and W4A4 -- each against its roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the layer on its own tokens (weak scaling, no collective on the data path);
+time is the max over ranks.  `--impl reference` times the CPU oracle on the
+host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "MXFP4 MoE GEMM TFLOP/s & weight GB/s vs roofline; quantize GB/s (1 B200)"
+L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_LAYER = {0: 6, 1: 8}   # W4A16: route x3, gate/up, down, combine; W4A4: + 2 quantize
+
+
+# ------------------------------------------------------------------ environment
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx_ = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        load = [v for v in sm if v > 0.5 * (max(mx_) if mx_ else 1)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx_) if mx_ else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workload set-up
+
+def layer_flops(T, k, H, I):
+    return 2.0 * T * k * (2 * I * H + H * I)
+
+
+def gpu_layer(cfg, dev, T=None):
+    """MoE layer inputs on the GPU; expert weights drawn per expert (seeded, fp32)
+    and quantized to MXFP4 by the library's own quantize kernel."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    x, logits = inputs.moe_activations(cfg, T)
+    E, H, I = cfg.E, cfg.H, cfg.I
+    w13c = torch.empty((E, 2 * I, H // 2), dtype=torch.uint8, device=dev)
+    w13s = torch.empty((E, 2 * I, H // 32), dtype=torch.uint8, device=dev)
+    w2c = torch.empty((E, H, I // 2), dtype=torch.uint8, device=dev)
+    w2s = torch.empty((E, H, I // 32), dtype=torch.uint8, device=dev)
+    for e in range(E):
+        w13, w2 = inputs.expert_weights(cfg, e)
+        mx.mxfp4_quantize(w13.to(dev), codes=w13c[e], scales=w13s[e])
+        mx.mxfp4_quantize(w2.to(dev), codes=w2c[e], scales=w2s[e])
+    torch.cuda.synchronize()
+    return dict(x=x, logits=logits, w=(w13c, w13s, w2c, w2s))
+
+
+def make_events(n):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    return evs
+
+
+def time_layer(L, cfg, mode, steps, warmup, dev, world=1, trace=True, flush=None):
+    """Device time of `steps` layer calls (inputs resident), L2 flushed before each.
+    Returns per-step ms, per-stage ms (gate/up, down, ...) and the outer wall."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    T = L["x"].shape[0]
+    xd, ld = L["x"].to(dev), L["logits"].to(dev)
+    out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((mx.moe_mxfp4_workspace_size(T, cfg.H, cfg.I, cfg.E, cfg.top_k, mode),),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev) if flush is None else flush
+    for _ in range(warmup):
+        flush.zero_()
+        mx.moe_mxfp4_mlp(xd, ld, cfg.top_k, *L["w"], mode=mode, out=out, ws=ws)
+    torch.cuda.synchronize()
+    assert mx.mxfp4_get_device_status() == 0
+    starts, ends = make_events(steps), make_events(steps)
+    stage = [make_events(5) for _ in range(steps)] if trace else None
+    outer0, outer1 = make_events(2)
+    barrier(world)
+    torch.cuda.synchronize()
+    outer0.record()
+    for i in range(steps):
+        flush.zero_()
+        if trace:
+            mx.mxfp4_set_trace_events(stage[i])
+        starts[i].record()
+        mx.moe_mxfp4_mlp(xd, ld, cfg.top_k, *L["w"], mode=mode, out=out, ws=ws)
+        ends[i].record()
+    outer1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    mx.mxfp4_set_trace_events(None)
+    assert mx.mxfp4_get_device_status() == 0
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    res = dict(step_ms=per_step, outer_ms=outer0.elapsed_time(outer1), out=out)
+    if trace:
+        names = ["route", "gate_up", "down", "combine"]
+        res["stage_ms"] = {n: statistics.mean(st[j].elapsed_time(st[j + 1]) for st in stage)
+                           for j, n in enumerate(names)}
+    return res
+
+
+def time_e2e(L, cfg, mode, steps, warmup, dev):
+    """Same layer through the public API with host buffers: pinned H2D of x and
+    the router logits, the call, D2H of the output -- all inside the timing."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    T = L["x"].shape[0]
+    hx = L["x"].pin_memory()
+    hl = L["logits"].pin_memory()
+    hout = torch.empty((T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(hx, device=dev)
+    ld = torch.empty_like(hl, device=dev)
+    out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((mx.moe_mxfp4_workspace_size(T, cfg.H, cfg.I, cfg.E, cfg.top_k, mode),),
+                     dtype=torch.uint8, device=dev)
+
+    def one():
+        xd.copy_(hx, non_blocking=True)
+        ld.copy_(hl, non_blocking=True)
+        mx.moe_mxfp4_mlp(xd, ld, cfg.top_k, *L["w"], mode=mode, out=out, ws=ws)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a, b = make_events(2)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, hx.numel() * 2 + hl.numel() * 4, hout.numel() * 2
+
+
+def time_kernel(fn, steps, warmup, dev, flush):
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    s, e = make_events(steps), make_events(steps)
+    for i in range(steps):
+        flush.zero_()
+        s[i].record()
+        fn()
+        e[i].record()
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in zip(s, e))
+
+
+# ------------------------------------------------------------------ breakdown lines
+
+def bench_quant(dev, pk, flush, steps=20, warmup=5):
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    x = inputs.quant_tensor().to(dev)
+    R, C = x.shape
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, C // 32), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x)
+    nbytes = R * C * 2 + R * C // 2 + R * C // 32
+    tq = time_kernel(lambda: mx.mxfp4_quantize(x, codes=codes, scales=scales), steps, warmup, dev, flush)
+    td = time_kernel(lambda: mx.mxfp4_dequantize(codes, scales, out=out), steps, warmup, dev, flush)
+    gq, gd = nbytes / tq / 1e6, nbytes / td / 1e6
+    return {"workload": f"bf16 [{R}, {C}] <-> MXFP4 (1% x50 outliers, 0.5% zero blocks)",
+            "bytes_per_call": nbytes,
+            "quantize": {"us": tq * 1e3, "gbs": gq, "frac_hbm": gq / pk["hbm"]},
+            "dequantize": {"us": td * 1e3, "gbs": gd, "frac_hbm": gd / pk["hbm"]}}
+
+
+def active_weight_bytes(cfg, logits):
+    ids = torch.topk(logits, cfg.top_k, dim=1).indices.unique().numel()
+    per_expert = (2 * cfg.I * cfg.H + cfg.H * cfg.I) * (0.5 + 1 / 32)
+    return ids, ids * per_expert
+
+
+def bench_moe_line(name, cfg, L, mode, dev, pk, flush, steps=10, warmup=3):
+    r = time_layer(L, cfg, mode, steps, warmup, dev, flush=flush)
+    ms = statistics.mean(r["step_ms"])
+    fl = layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I)
+    n_act, wbytes = active_weight_bytes(cfg, L["logits"])
+    st = r["stage_ms"]
+    line = {"workload": f"{name}: T={cfg.T} E={cfg.E} top-{cfg.top_k} H={cfg.H} I={cfg.I} "
+                        f"{'W4A4' if mode else 'W4A16'}",
+            "us_per_layer": ms * 1e3, "tflops": fl / ms / 1e9, "tokens_per_s": cfg.T / ms * 1e3,
+            "active_experts": n_act, "weight_gbs": wbytes / ms / 1e6,
+            "frac_hbm_weights": wbytes / ms / 1e6 / pk["hbm"],
+            "frac_bf16": fl / ms / 1e9 / pk["bf16"],
+            "stage_us": {k: v * 1e3 for k, v in st.items()}}
+    gu_w = 2 * cfg.I * cfg.H * (0.5 + 1 / 32) * n_act
+    dn_w = cfg.H * cfg.I * (0.5 + 1 / 32) * n_act
+    line["gate_up"] = {"weight_gbs": gu_w / st["gate_up"] / 1e6,
+                       "frac_hbm": gu_w / st["gate_up"] / 1e6 / pk["hbm"],
+                       "tflops": fl * 2 / 3 / st["gate_up"] / 1e9,
+                       "frac_bf16": fl * 2 / 3 / st["gate_up"] / 1e9 / pk["bf16"]}
+    line["down"] = {"weight_gbs": dn_w / st["down"] / 1e6,
+                    "frac_hbm": dn_w / st["down"] / 1e6 / pk["hbm"],
+                    "tflops": fl / 3 / st["down"] / 1e9,
+                    "frac_bf16": fl / 3 / st["down"] / 1e9 / pk["bf16"]}
+    return line
+
+
+def breakdown(dev, pk, flush):
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    bd = {"quant": bench_quant(dev, pk, flush)}
+    cfg = inputs.MOE_CONFIGS["moe_decode"]
+    L = gpu_layer(cfg, dev)
+    bd["moe_decode"] = bench_moe_line("moe_decode", cfg, L, mx.W4A16, dev, pk, flush, steps=20)
+    del L
+    cfg = inputs.MOE_CONFIGS["moe_120b"]
+    L = gpu_layer(cfg, dev)
+    bd["moe_120b_w4a16"] = bench_moe_line("moe_120b", cfg, L, mx.W4A16, dev, pk, flush)
+    bd["moe_120b_w4a4"] = bench_moe_line("moe_120b", cfg, L, mx.W4A4, dev, pk, flush)
+    del L
+    torch.cuda.empty_cache()
+    return bd
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_weights(cfg):
+    import oracle
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    E, H, I = cfg.E, cfg.H, cfg.I
+    w13c = np.empty((E, 2 * I, H // 2), np.uint8)
+    w13s = np.empty((E, 2 * I, H // 32), np.uint8)
+    w2c = np.empty((E, H, I // 2), np.uint8)
+    w2s = np.empty((E, H, I // 32), np.uint8)
+    for e in range(E):
+        w13, w2 = inputs.expert_weights(cfg, e)
+        w13c[e], w13s[e] = oracle.quantize(w13.numpy(), oracle.FLOOR)
+        w2c[e], w2s[e] = oracle.quantize(w2.numpy(), oracle.FLOOR)
+    return w13c, w13s, w2c, w2s
+
+
+def oracle_run(cfg, W, tokens):
+    import oracle
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    x, logits = inputs.moe_activations(cfg)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    oracle.moe_mlp(xb, logits.numpy(), cfg.top_k, *W, tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def cpu_threads():
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, n_tokens=16, seed=0):
+    """The oracle, as it stands, on a seeded sample of the workload's tokens."""
+    W = oracle_weights(cfg)
+    g = torch.Generator().manual_seed(seed)
+    tok = torch.randperm(cfg.T, generator=g)[:n_tokens].numpy()
+    dt = oracle_run(cfg, W, tok)
+    fl = layer_flops(n_tokens, cfg.top_k, cfg.H, cfg.I)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n_tokens} seeded tokens of the {cfg.T}-token layer (all their top-{cfg.top_k} "
+                      f"experts: fp64 dequantize + fp64 matmuls), {dt:.1f} s wall"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, K timed steps of one token each."""
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    if rank != 0:
+        return
+    cfg = inputs.MOE_CONFIGS["moe_prefill"]
+    W = oracle_weights(cfg)
+    g = torch.Generator().manual_seed(1234)
+    tok = torch.randperm(cfg.T, generator=g).numpy()
+    for i in range(args.warmup):
+        oracle_run(cfg, W, tok[i:i + 1])
+    times = [oracle_run(cfg, W, tok[args.warmup + i:args.warmup + i + 1]) for i in range(args.steps)]
+    dt = sum(times)
+    fl = layer_flops(args.steps, cfg.top_k, cfg.H, cfg.I)
+    v = fl / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(cfg),
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": "each step: 1 seeded token of the 8192-token prefill layer "
+                                       "(its 4 experts dequantized in fp64, fp64 matmuls)"},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg):
+    return {"workload": f"moe_prefill: gpt-oss-20b-shaped MoE expert-MLP layer, T={cfg.T} tokens, "
+                        f"{cfg.E} experts, top-{cfg.top_k}, +2.0 router bias on experts 0-3, "
+                        "MXFP4 weights, W4A16",
+            "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.top_k,
+            "flops_per_step": layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I),
+            "l2": "256 MiB buffer written before every step (outside the per-step events); "
+                  "weights 423 MB > 126 MB L2",
+            "parallelism": "replicas (one layer per GPU, no collective)"}
+
+
+def traffic_record(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        recs = json.load(f)
+    src = os.path.join(ROOT, "moe_expert_gemm_mxfp4_b200", "csrc", "gemm.cu")
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    r = recs.get(f"{kernel}|{workload}")
+    if not r or r.get("source_sha256_16") != h:
+        return None
+    return r.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T of the prefill workload (profiling runs on a smaller case)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    mx._lib.load()   # fails loudly if the library is missing
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    pk = peaks()
+    cfg = inputs.MOE_CONFIGS["moe_prefill"]
+    if args.tokens:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, T=args.tokens)
+    L = gpu_layer(cfg, dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler.start()
+    r = time_layer(L, cfg, mx.W4A16, args.steps, args.warmup, dev, world=world, flush=flush)
+    clocks = sampler.stop()
+
+    fl = layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I)
+    step_ms = statistics.mean(r["step_ms"])
+    total_ms = max_over_ranks(sum(r["step_ms"]), world)
+    value = world * args.steps * fl / total_ms / 1e9
+    st = r["stage_ms"]
+    gu_flops = 2.0 * cfg.T * cfg.top_k * 2 * cfg.I * cfg.H
+    achieved = gu_flops / st["gate_up"] / 1e9
+    roof = {"kernel": "grouped_w4a16_kernel<128, SWIGLU> (gate/up projection + SwiGLU)",
+            "bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+            "frac": achieved / pk["bf16"],
+            "peak_source": f"{pk['source']} bf16 dense (burst; timed region < 1 s)",
+            "flops_per_launch": gu_flops,
+            "traffic": traffic_record("grouped_w4a16_kernel_swiglu", "moe_prefill")}
+
+    if rank != 0:
+        barrier(world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    e2e_ms, h2d, d2h = time_e2e(L, cfg, mx.W4A16, max(3, args.steps // 2), 3, dev)
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded torch CPU generator; weights ~N(0,0.02) quantized to MXFP4)",
+            "config": workload_config(cfg),
+            "tokens_per_s": world * args.steps * cfg.T / total_ms * 1e3,
+            "stage_us": {k: v * 1e3 for k, v in st.items()},
+            "roofline": roof,
+            "e2e": {"value": fl / e2e_ms / 1e9, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": KERNELS_PER_LAYER[0] * args.steps,
+            "clocks": clocks}
+    del L
+    torch.cuda.empty_cache()
+    if not args.no_breakdown and world == 1:
+        line["breakdown"] = breakdown(dev, pk, flush)
+    if not args.no_cpu and world == 1:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(world)
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -93,7 +93,8 @@ MXFP4_API mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* sca
 /* ---------------------------------------------------------------- GEMM
  * y [M, N] bf16 = x [M, K] bf16 . dequant(W)^T, W = MXFP4 codes [N, K/2] +
  * scales [N, K/32]; fp32 accumulation, one rounding to bf16 at the end.
- * Requires K % 64 == 0; any M >= 1, N >= 1.  Workspace: W4A16 needs none
+ * Requires K % 64 == 0 and K <= 11712 (the block scales of a 128-row weight tile
+ * are staged whole in shared memory); any M >= 1, N >= 1.  Workspace: W4A16 needs none
  * (ws may be NULL); W4A4 needs mxfp4_gemm_workspace_size() bytes (the quantized x). */
 MXFP4_API mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K,
                         const uint8_t* w_codes, const uint8_t* w_scales, int64_t N,
@@ -127,7 +128,7 @@ MXFP4_API size_t moe_mxfp4_route_workspace_size(int64_t T, int64_t E, int32_t to
  *   out[t] = bf16( sum_j y_tj ) in slot order (deterministic; no atomics).
  * x bf16 [T, H]; router_logits fp32 [T, E]; w13 codes uint8 [E, 2I, H/2] +
  * scales uint8 [E, 2I, H/32]; w2 codes uint8 [E, H, I/2] + scales [E, H, I/32];
- * out bf16 [T, H].  Requires H % 64 == 0, I % 64 == 0, 1 <= top_k <= min(E, 8),
+ * out bf16 [T, H].  Requires H % 64 == 0, I % 64 == 0, H, I <= 11712, 1 <= top_k <= min(E, 8),
  * E <= 256, T*top_k < 2^31.  ws must hold moe_mxfp4_workspace_size() bytes
  * (routing tables and the per-pair activations h / y). */
 MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,
@@ -138,6 +139,17 @@ MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,
                            void* stream);
 MXFP4_API size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k,
                                 mxfp4_mode mode);
+
+/* ---------------------------------------------------------------- tracing
+ * Optional stage timing for the calling host thread.  `events` points to
+ * `n_events` cudaEvent_t handles (passed as void*) created by the caller; while
+ * set, moe_mxfp4_mlp records events[i] on its stream at stage boundary i:
+ *   0 start, 1 after routing + gather (W4A4: + activation quantization),
+ *   2 after the gate/up GEMM + SwiGLU, 3 after the down GEMM (W4A4: + the
+ *   quantization of h before it), 4 after the combine.
+ * Boundaries beyond n_events are skipped.  Pass NULL / 0 to disable.  The
+ * pointer array must stay valid while tracing is on.  Never fails. */
+MXFP4_API void mxfp4_set_trace_events(void* const* events, int n_events);
 
 /* ---------------------------------------------------------------- status
  * Synchronizes `stream`, then returns and clears the current device's device-side

@@ -24,7 +24,8 @@ from ._lib import (Mxfp4Error, Mxfp4LibraryMissing, SCALE_CEIL, SCALE_FLOOR, W4A
 __all__ = [
     "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_gemm_workspace_size",
     "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
-    "moe_mxfp4_workspace_size", "mxfp4_get_device_status", "Mxfp4Error", "Mxfp4LibraryMissing",
+    "moe_mxfp4_workspace_size", "mxfp4_get_device_status", "mxfp4_set_trace_events",
+    "Mxfp4Error", "Mxfp4LibraryMissing",
     "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
 ]
 
@@ -151,3 +152,22 @@ def moe_mxfp4_mlp(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13_codes, 
 def mxfp4_get_device_status(stream=None) -> int:
     """Synchronize the stream and return (and clear) the device status word."""
     return int(_lib.load().mxfp4_get_device_status(_stream(stream)))
+
+
+_trace_keepalive = None
+
+
+def mxfp4_set_trace_events(events=None):
+    """Record the given torch.cuda.Event objects (already created: recorded once)
+    at the stage boundaries of subsequent moe_mxfp4_mlp calls on this thread
+    (0 start, 1 routed + gathered, 2 gate/up done, 3 down done, 4 combined).
+    ``None`` turns tracing off."""
+    global _trace_keepalive
+    lib = _lib.load()
+    if not events:
+        _trace_keepalive = None
+        lib.mxfp4_set_trace_events(None, 0)
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _trace_keepalive = arr
+    lib.mxfp4_set_trace_events(ctypes.cast(arr, ctypes.c_void_p), len(events))

@@ -56,6 +56,7 @@ _SIGS = {
                                      ctypes.c_int, _vp, _sz, _vp]),
     "moe_mxfp4_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, ctypes.c_int]),
     "mxfp4_get_device_status": (ctypes.c_int, [_vp]),
+    "mxfp4_set_trace_events": (None, [_vp, ctypes.c_int]),
     "mxfp4_last_cuda_error": (ctypes.c_int, []),
     "mxfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }

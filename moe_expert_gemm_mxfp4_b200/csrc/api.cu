@@ -17,6 +17,14 @@ __device__ unsigned g_mxfp4_status;
 namespace {
 
 thread_local int tl_last_cuda_error = 0;
+thread_local void* const* tl_trace_events = nullptr;
+thread_local int tl_trace_n = 0;
+
+// Stage boundary i of a traced call (no-op unless tracing is on).
+void trace_mark(int i, cudaStream_t s) {
+    if (tl_trace_events && i < tl_trace_n && tl_trace_events[i])
+        cudaEventRecord(static_cast<cudaEvent_t>(tl_trace_events[i]), s);
+}
 
 constexpr int kMaxDevices = 64;
 
@@ -180,6 +188,11 @@ const char* mxfp4_status_string(mxfp4_status s) {
 
 int mxfp4_last_cuda_error(void) { return tl_last_cuda_error; }
 
+void mxfp4_set_trace_events(void* const* events, int n_events) {
+    tl_trace_events = n_events > 0 ? events : nullptr;
+    tl_trace_n = n_events > 0 ? n_events : 0;
+}
+
 mxfp4_status mxfp4_get_device_status(void* stream) {
     DeviceInfo* d = nullptr;
     mxfp4_status st = device_info(&d);
@@ -243,7 +256,7 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     if (M <= 0 || K <= 0 || N <= 0) return MXFP4_ERR_INVALID_ARG;
     if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
     if (K % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
-    if (M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) || K >= (int64_t{1} << 24))
+    if (M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) || K > mx::max_gemm_k())
         return MXFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x_bf16) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y_bf16))
         return MXFP4_ERR_MISALIGNED;
@@ -335,7 +348,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     if (H <= 0 || I <= 0) return MXFP4_ERR_INVALID_ARG;
     if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
     if (H % 64 != 0 || I % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
-    if (H >= (int64_t{1} << 24) || I >= (int64_t{1} << 24)) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (H > mx::max_gemm_k() || I > mx::max_gemm_k()) return MXFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x_bf16) || !aligned16(router_logits) || !aligned16(w13_codes) ||
         !aligned16(w13_scales) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
         !aligned16(out_bf16))
@@ -350,6 +363,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     const int64_t P = T * top_k;
     cudaError_t e;
 
+    trace_mark(0, s);
     const void* x_src = x_bf16;
     if (mode == MXFP4_W4A4) {   // activations on the MXFP4 grid, rows along H
         if ((e = mx::launch_qdq_bf16(x_bf16, T, H, w.y_sorted, d->sm_count, s)) != cudaSuccess)
@@ -361,6 +375,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
                               d->sm_count, s)) != cudaSuccess)
         return cuda_fail(e);
 
+    trace_mark(1, s);
     const int nt = mx::pick_token_tile(P, E);
     const int64_t tok_tiles = (P + nt - 1) / nt + E;
 
@@ -386,6 +401,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
                                      gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
         return cuda_fail(e);
 
+    trace_mark(2, s);
     if (mode == MXFP4_W4A4) {   // h on the MXFP4 grid, rows along I (in place)
         if ((e = mx::launch_qdq_bf16(w.h, P, I, w.h, d->sm_count, s)) != cudaSuccess)
             return cuda_fail(e);
@@ -407,10 +423,12 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
                                      gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
         return cuda_fail(e);
 
+    trace_mark(3, s);
     // deterministic combine in slot order
     if ((e = mx::launch_combine(w.y_sorted, w.inv, T, top_k, H, out_bf16, d->sm_count, s)) !=
         cudaSuccess)
         return cuda_fail(e);
+    trace_mark(4, s);
     return MXFP4_OK;
 }
 

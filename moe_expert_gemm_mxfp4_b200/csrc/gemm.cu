@@ -12,9 +12,11 @@
 // and "Zero-Build Kernels from the Hub").
 //
 // Data flow (one persistent CTA per SM, 16 warps):
-//   warp 0        TMA producer: per 64-wide K stage, the packed codes of 128
-//                 weight rows (32 B per row, 32B-swizzled) and the bf16
-//                 activation tile [NT rows x 64] (128B-swizzled) -> smem ring.
+//   warp 0        TMA producer: per tile, the block scales of its 128 weight
+//                 rows (bulk copy, double-buffered across tiles); per 64-wide K
+//                 stage, the packed codes of the 128 rows (32 B per row,
+//                 32B-swizzled) and the bf16 activation tile [NT x 64]
+//                 (128B-swizzled) -> smem ring.
 //   warps 4..11   two dequant warpgroups (alternate stages): each thread owns
 //                 one weight row; codes -> bf16 through a 256-entry shared LUT
 //                 (lane-replicated, conflict-free) times the block scale 2^(S-127)
@@ -25,7 +27,8 @@
 //                 N = NT tokens, K = 16 per instruction, A from TMEM, B from
 //                 smem, D (fp32) in TMEM, double-buffered across tiles.
 //   warps 12..15  epilogue: tcgen05.ld of the accumulator, fused epilogue,
-//                 bf16 stores.
+//                 stores.
+// TMEM: columns [0, 2*NT) the two accumulators, [256, 512) eight A slots.
 // Every mbarrier wait is time-bounded (MXFP4_ERR_TIMEOUT in the status word).
 #include "common.cuh"
 #include "internal.h"
@@ -37,29 +40,42 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kBM = 128;            // weight rows per tile (MMA M)
 constexpr int kBK = 64;             // K per pipeline stage
-constexpr int kASlots = 4;          // TMEM A-operand slots (32 columns each)
+constexpr int kASlots = 8;          // TMEM A-operand slots (32 columns each)
 constexpr int kACol0 = 256;         // first TMEM column of the A slots
 constexpr int kCodeBytes = kBM * kBK / 2;
 constexpr int kLutBytes = 256 * 256;
 constexpr int kMaxGroups = 256;
+constexpr int kXbufBytes = 2 * 2 * 32 * 16 * 4;
+constexpr int kSmemLimit = 227 * 1024;
 
 template <int NT>
 struct Cfg {
     static constexpr int kActBytes = NT * kBK * 2;
     static constexpr int kStageBytes = kCodeBytes + kActBytes;
-    static constexpr int kStages = NT <= 32 ? 10 : (NT == 64 ? 8 : 5);
-    static constexpr int kXbufBytes = 2 * 2 * 32 * 16 * 4;
-    static constexpr int kStagesOff = kLutBytes;
-    static constexpr int kXbufOff = kStagesOff + kStages * kStageBytes;
-    static constexpr int kBarOff = kXbufOff + kXbufBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 * kASlots + 4 + 1;
-    static constexpr int kTstartOff = kBarOff + kNumBars * 8;
-    static constexpr int kOffOff = kTstartOff + (kMaxGroups + 1) * 4;
-    static constexpr int kMiscOff = kOffOff + (kMaxGroups + 1) * 4;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;   // + alignment slack
+    static constexpr int kMaxStages = NT == 16 ? 16 : (NT == 32 ? 12 : (NT == 64 ? 8 : 5));
     static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-B alignment");
     static_assert(2 * NT <= kACol0, "accumulators overlap the A slots");
 };
+
+// Shared-memory layout, identical on host (sizing) and device.
+struct Layout {
+    int stages_off, scales_off, scale_bytes, xbuf_off, bar_off, tstart_off, off_off, misc_off, total;
+};
+
+__host__ __device__ inline Layout make_layout(int stage_bytes, int stages, int K) {
+    Layout L;
+    L.stages_off = kLutBytes;
+    L.scales_off = L.stages_off + stages * stage_bytes;
+    L.scale_bytes = ((kBM * (K / 32)) + 127) / 128 * 128;
+    L.xbuf_off = L.scales_off + 2 * L.scale_bytes;
+    L.bar_off = L.xbuf_off + kXbufBytes;
+    const int n_bars = 2 * 16 + 2 * kASlots + 4 + 4 + 1;
+    L.tstart_off = L.bar_off + n_bars * 8;
+    L.off_off = L.tstart_off + (kMaxGroups + 1) * 4;
+    L.misc_off = L.off_off + (kMaxGroups + 1) * 4;
+    L.total = L.misc_off + 16 + 1024;   // + slack for the 1024-B alignment of the base
+    return L;
+}
 
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -73,6 +89,12 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -81,21 +103,15 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint16_t ldg_nc_u16(const uint8_t* p) {
-    uint16_t v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-    return v;
-}
-
 // 16 code bytes (32 weights of one K block) -> 16 bf16x2 words.
 // Fast path (S in [2, 254]): LUT value times 2^(S-127) as one bf16x2 multiply,
 // exact because both factors and the product are normal bf16 numbers (or the
 // product overflows to Inf, as round-to-nearest-even does).  Otherwise the
 // exact fp32 route (subnormal results for S <= 1, NaN for S = 255).
+// LUT entry (b, lane) sits at lut_base + b * 256 + lane * 4; lut_lane is
+// lut_base + lane * 4 and prmt places code byte j of a word at bits 8..15.
 __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lut_lane,
                                                 uint32_t* out) {
-    // LUT entry (b, lane) sits at lut_base + b * 256 + lane * 4; lut_lane is
-    // lut_base + lane * 4 and prmt places the code byte at bits 8..15.
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     if (S - 2u <= 252u) {
         const uint32_t sf = S * 0x00800080u;      // bf16x2 {2^(S-127), 2^(S-127)}
@@ -116,7 +132,7 @@ __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lu
     }
 }
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void store_bf16(void* out, int64_t idx, float v) {
     reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
@@ -148,37 +164,59 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const int* s_tstart, cons
     return ti;
 }
 
+// Copy `rows` consecutive rows of block scales (kb bytes each) from global to
+// shared: the 16-byte multiple with one bulk copy (counted on `bar`), the tail
+// with plain loads.  Returns the bulk byte count.
+__device__ __forceinline__ uint32_t stage_scales(uint8_t* dst, const uint8_t* src, int rows, int kb,
+                                                 uint64_t* bar) {
+    const uint32_t bytes = static_cast<uint32_t>(rows * kb);
+    const uint32_t bulk = bytes & ~15u;
+    if (bulk) bulk_load(dst, src, bulk, bar);
+    if (bulk < bytes) {
+        for (uint32_t i = bulk; i < bytes; ++i) dst[i] = src[i];
+        // order these generic-proxy writes before later bulk copies into the buffer
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    return bulk;
+}
+
 template <int NT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
     using C = Cfg<NT>;
+    const int S_ = args.stages;
+    const Layout Ly = make_layout(C::kStageBytes, S_, args.K);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-    uint8_t* stages = smem + C::kStagesOff;
-    float* xbuf = reinterpret_cast<float*>(smem + C::kXbufOff);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + C::kStages;
-    uint64_t* afull = bars + 2 * C::kStages;
-    uint64_t* aempty = afull + kASlots;
-    uint64_t* accfull = aempty + kASlots;
-    uint64_t* accempty = accfull + 2;
-    uint64_t* drain = accempty + 2;
-    int* s_tstart = reinterpret_cast<int*>(smem + C::kTstartOff);
-    int* s_off = reinterpret_cast<int*>(smem + C::kOffOff);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
-    volatile int* s_never = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);   // stays 0
+    uint8_t* stages = smem + Ly.stages_off;
+    uint8_t* scales = smem + Ly.scales_off;
+    float* xbuf = reinterpret_cast<float*>(smem + Ly.xbuf_off);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bar_off);
+    uint64_t* full = bars;                 // [16] stage filled (TMA tx)
+    uint64_t* empty = bars + 16;           // [16] stage consumed (MMA commit)
+    uint64_t* afull = bars + 32;           // [8]  A slot written (128 dequant threads)
+    uint64_t* aempty = afull + kASlots;    // [8]  A slot consumed (MMA commit)
+    uint64_t* accfull = aempty + kASlots;  // [2]  accumulator ready (MMA commit)
+    uint64_t* accempty = accfull + 2;      // [2]  accumulator drained (128 epilogue threads)
+    uint64_t* sfull = accempty + 2;        // [2]  tile scales staged (tx)
+    uint64_t* sempty = sfull + 2;          // [2]  tile scales no longer needed (MMA commit)
+    uint64_t* drain = sempty + 2;
+    int* s_tstart = reinterpret_cast<int*>(smem + Ly.tstart_off);
+    int* s_off = reinterpret_cast<int*>(smem + Ly.off_off);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc_off);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Ly.misc_off + 4);
+    volatile int* s_never = reinterpret_cast<volatile int*>(smem + Ly.misc_off + 8);   // stays 0
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = args.offsets ? args.G : 1;
+    const int kb = args.K / 32;            // scale bytes per weight row
 
     // ---------------- set-up
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < S_; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -189,6 +227,8 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accfull[b], 1);
             mbar_init(&accempty[b], 128);
+            mbar_init(&sfull[b], 1);
+            mbar_init(&sempty[b], 1);
         }
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -229,33 +269,52 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     if (warp == 0) {
         // ---------------- TMA producer
         if (lane == 0) {
-            int kit = 0;
+            int kit = 0, lt = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
                 const TileInfo ti = decode_tile<NT>(t, s_tstart, s_off, G);
+                // block scales of the tile's weight rows, in the smem row order of the codes
+                const int sb = lt & 1;
+                if (!mbar_wait(&sempty[sb], ((lt >> 1) & 1) ^ 1, s_abort)) { ok = false; break; }
+                uint8_t* sdst = scales + sb * Ly.scale_bytes;
+                const uint8_t* gsc = args.w_scales + static_cast<int64_t>(ti.g) * args.rows_w * kb;
+                uint32_t tx = 0;
+                if (MODE == EPI_SWIGLU) {
+                    tx += stage_scales(sdst, gsc + static_cast<int64_t>(ti.f * 64) * kb, 64, kb, &sfull[sb]);
+                    tx += stage_scales(sdst + 64 * kb, gsc + static_cast<int64_t>(args.I + ti.f * 64) * kb,
+                                       64, kb, &sfull[sb]);
+                } else {
+                    const int rows = min(kBM, args.rows_w - ti.f * kBM);
+                    tx += stage_scales(sdst, gsc + static_cast<int64_t>(ti.f * kBM) * kb, rows, kb, &sfull[sb]);
+                }
+                mbar_arrive_expect_tx(&sfull[sb], tx);
                 for (int ks = 0; ks < nk; ++ks, ++kit) {
-                    const int st = kit % C::kStages;
-                    const uint32_t ph = (kit / C::kStages) & 1;
+                    const int st = kit % S_;
+                    const uint32_t ph = (kit / S_) & 1;
                     if (!mbar_wait(&empty[st], ph ^ 1, s_abort)) { ok = false; break; }
-                    uint8_t* sb = stages + st * C::kStageBytes;
+                    uint8_t* sb_ = stages + st * C::kStageBytes;
                     mbar_arrive_expect_tx(&full[st], C::kStageBytes);
                     if (MODE == EPI_SWIGLU) {
-                        tma_load_3d(sb, &tmap_w, &full[st], ks * 32, ti.f * 64, ti.g);
-                        tma_load_3d(sb + 64 * 32, &tmap_w, &full[st], ks * 32, args.I + ti.f * 64, ti.g);
+                        tma_load_3d(sb_, &tmap_w, &full[st], ks * 32, ti.f * 64, ti.g);
+                        tma_load_3d(sb_ + 64 * 32, &tmap_w, &full[st], ks * 32, args.I + ti.f * 64, ti.g);
                     } else {
-                        tma_load_3d(sb, &tmap_w, &full[st], ks * 32, ti.f * kBM, ti.g);
+                        tma_load_3d(sb_, &tmap_w, &full[st], ks * 32, ti.f * kBM, ti.g);
                     }
-                    tma_load_2d(sb + kCodeBytes, &tmap_x, &full[st], ks * kBK, ti.row0);
+                    tma_load_2d(sb_ + kCodeBytes, &tmap_x, &full[st], ks * kBK, ti.row0);
                 }
             }
             if (!ok) {
                 *s_abort = 1;
                 record_status(args.status, MXFP4_ERR_TIMEOUT);
                 // let the copies already issued land before the CTA exits
-                const int n_inflight = kit < C::kStages ? kit : C::kStages;
+                const int n_inflight = kit < S_ ? kit : S_;
                 for (int i = 1; i <= n_inflight; ++i) {
                     const int k2 = kit - i;
-                    mbar_wait(&full[k2 % C::kStages], (k2 / C::kStages) & 1, s_never);
+                    mbar_wait(&full[k2 % S_], (k2 / S_) & 1, s_never);
+                }
+                for (int i = 1; i <= 2 && i <= lt + 1; ++i) {
+                    const int l2 = lt + 1 - i;
+                    mbar_wait(&sfull[l2 & 1], (l2 >> 1) & 1, s_never);
                 }
             }
         }
@@ -271,9 +330,9 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * NT;
                 for (int ks = 0; ks < nk; ++ks, ++kit) {
-                    const int st = kit % C::kStages;
+                    const int st = kit % S_;
                     const int as = kit % kASlots;
-                    if (!mbar_wait(&full[st], (kit / C::kStages) & 1, s_abort) ||
+                    if (!mbar_wait(&full[st], (kit / S_) & 1, s_abort) ||
                         !mbar_wait(&afull[as], (kit / kASlots) & 1, s_abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t b_base = smem_u32(stages + st * C::kStageBytes + kCodeBytes);
@@ -287,6 +346,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 }
                 if (!ok) break;
                 tc_commit(&accfull[acc]);
+                tc_commit(&sempty[lt & 1]);
             }
             if (!ok) {
                 *s_abort = 1;
@@ -301,33 +361,33 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         const int d = (warp - 4) >> 2;        // 0 or 1: even or odd stages
         const int q = warp & 3;               // TMEM lane quarter
         const uint32_t lut_lane = smem_u32(lut) + lane * 4;
-        const int kb = args.K / 32;
-        int kit = 0;
+        int srow;
+        if (MODE == EPI_SWIGLU) {
+            const int half = q >> 1, up = q & 1;
+            srow = up * 64 + half * 32 + lane;  // lanes: gate 0-31 | up 0-31 | gate 32-63 | up 32-63
+        } else {
+            srow = q * 32 + lane;
+        }
+        const uint32_t sw = (static_cast<uint32_t>(srow) >> 2) & 1u;
+        int kit = 0, lt = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
             const TileInfo ti = decode_tile<NT>(t, s_tstart, s_off, G);
-            int srow, wrow;
-            if (MODE == EPI_SWIGLU) {
-                const int half = q >> 1, up = q & 1;
-                srow = up * 64 + half * 32 + lane;
-                wrow = up * args.I + ti.f * 64 + half * 32 + lane;
-            } else {
-                srow = q * 32 + lane;
-                wrow = ti.f * kBM + srow;
-            }
-            const bool valid = wrow < args.rows_w;
-            const uint8_t* sc_row =
-                args.w_scales + (static_cast<int64_t>(ti.g) * args.rows_w + (valid ? wrow : 0)) * kb;
-            const uint32_t sw = (static_cast<uint32_t>(srow) >> 2) & 1u;
+            const bool valid = MODE == EPI_SWIGLU || ti.f * kBM + srow < args.rows_w;
+            const uint32_t sc_row = smem_u32(scales + (lt & 1) * Ly.scale_bytes) + srow * kb;
+            bool scales_ready = false;
             for (int ks = 0; ks < nk; ++ks, ++kit) {
                 if ((kit & 1) != d) continue;
-                const int st = kit % C::kStages;
+                const int st = kit % S_;
                 const int as = kit % kASlots;
-                const uint32_t sc = valid ? ldg_nc_u16(sc_row + 2 * ks) : 0x7F7Fu;
-                const bool got = mbar_wait(&full[st], (kit / C::kStages) & 1, s_abort) &&
-                                 mbar_wait(&aempty[as], ((kit / kASlots) & 1) ^ 1, s_abort);
+                bool got = mbar_wait(&full[st], (kit / S_) & 1, s_abort) &&
+                           mbar_wait(&aempty[as], ((kit / kASlots) & 1) ^ 1, s_abort);
+                if (!scales_ready)
+                    got = got && mbar_wait(&sfull[lt & 1], (lt >> 1) & 1, s_abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+                scales_ready = true;
                 tc_fence_after();
+                const uint32_t sc = valid ? lds_u16(sc_row + 2 * ks) : 0x7F7Fu;
                 const uint32_t row_addr = smem_u32(stages + st * C::kStageBytes) + srow * 32;
                 const uint4 c0 = lds128(row_addr + ((0u ^ sw) << 4));
                 const uint4 c1 = lds128(row_addr + ((1u ^ sw) << 4));
@@ -416,14 +476,19 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
 }
 
 template <int NT, int MODE>
-cudaError_t launch_nt(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int grid,
+cudaError_t launch_nt(const CUtensorMap& tw, const CUtensorMap& tx, GemmArgs a, int grid,
                       cudaStream_t stream) {
     using C = Cfg<NT>;
+    // deepest ring that fits next to the LUT, the scale buffers and the rest
+    int stages = C::kMaxStages;
+    while (stages > 2 && make_layout(C::kStageBytes, stages, a.K).total > kSmemLimit) --stages;
+    const Layout L = make_layout(C::kStageBytes, stages, a.K);
+    if (stages < 3 || L.total > kSmemLimit) return cudaErrorInvalidConfiguration;
+    a.stages = stages;
     auto kern = grouped_w4a16_kernel<NT, MODE>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           C::kSmemBytes);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tw, tx, a);
+    kern<<<grid, kThreads, L.total, stream>>>(tw, tx, a);
     return cudaGetLastError();
 }
 
@@ -446,6 +511,14 @@ int pick_token_tile(int64_t rows, int64_t groups) {
     if (avg <= 32) return 32;
     if (avg <= 64) return 64;
     return 128;
+}
+
+// Largest K the kernel accepts (its tile's block scales must fit in shared memory
+// next to a 3-stage ring at the largest token tile).
+int64_t max_gemm_k() {
+    int64_t k = 64;
+    while (make_layout(Cfg<128>::kStageBytes, 3, static_cast<int>(k + 64)).total <= kSmemLimit) k += 64;
+    return k;
 }
 
 // Host launcher.  `tmap_w` covers the codes as a 3-D tensor {K/2, rows_w, G}

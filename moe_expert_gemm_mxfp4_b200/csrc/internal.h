@@ -25,6 +25,7 @@ struct GemmArgs {
     int n_valid_feat;          // valid output columns
     const float* row_w;        // WEIGHTED: per-row scalar
     unsigned* status;          // device status word
+    int stages;                // smem pipeline depth (set by launch_grouped_gemm)
 };
 
 cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t cols,
@@ -42,6 +43,7 @@ cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, i
 cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, int top_k,
                            int64_t H, void* out, int sm_count, cudaStream_t stream);
 int pick_token_tile(int64_t rows, int64_t groups);
+int64_t max_gemm_k();   // largest contraction length the grouped GEMM accepts
 cudaError_t launch_grouped_gemm(int mode, int nt, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream);
