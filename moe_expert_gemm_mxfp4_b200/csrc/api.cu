@@ -89,8 +89,9 @@ EncodeTiledFn encode_fn() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Packed codes of G groups as a 3-D tensor {K/2 bytes, rows, G}; box {32, box_rows, 1};
-// 32-byte swizzle (conflict-free 16-B reads of one row per thread).
+// Packed codes of G groups as a 3-D tensor {K/2 bytes, rows, G}; box {128, box_rows, 1}
+// (128 B = 256 K values of each row per copy); 128-byte swizzle (conflict-free 16-B
+// reads of one row per thread).
 mxfp4_status encode_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t K, int64_t rows,
                               int64_t G, int box_rows) {
     EncodeTiledFn fn = encode_fn();
@@ -99,10 +100,10 @@ mxfp4_status encode_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t K, i
                                 static_cast<cuuint64_t>(G)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2),
                                    static_cast<cuuint64_t>(rows * (K / 2))};
-    const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(codes), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
 }
@@ -273,10 +274,10 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
         if (e != cudaSuccess) return cuda_fail(e);
         xa = ws;
     }
-    const int nt = mx::pick_token_tile(M, 1);
+    const mx::TokenTiling tiling = mx::pick_token_tiling(M, 1);
     CUtensorMap tw, tx;
     if ((st = encode_codes_map(&tw, w_codes, K, N, 1, 128)) != MXFP4_OK) return st;
-    if ((st = encode_act_map(&tx, xa, K, M, nt)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, xa, K, M, tiling.nt)) != MXFP4_OK) return st;
     mx::GemmArgs a{};
     a.w_scales = w_scales;
     a.offsets = nullptr;
@@ -291,8 +292,9 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     a.n_valid_feat = static_cast<int>(N);
     a.row_w = nullptr;
     a.status = d->status;
-    const int64_t tiles = ((M + nt - 1) / nt) * a.n_ftiles;
-    cudaError_t e = mx::launch_grouped_gemm(mx::EPI_PLAIN, nt, tw, tx, a, gemm_grid(d, tiles), s);
+    const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
+    const int64_t tiles = ((M + tile_rows - 1) / tile_rows) * a.n_ftiles;
+    cudaError_t e = mx::launch_grouped_gemm(mx::EPI_PLAIN, tiling, tw, tx, a, gemm_grid(d, tiles), s);
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
@@ -376,13 +378,14 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
         return cuda_fail(e);
 
     trace_mark(1, s);
-    const int nt = mx::pick_token_tile(P, E);
-    const int64_t tok_tiles = (P + nt - 1) / nt + E;
+    const mx::TokenTiling tiling = mx::pick_token_tiling(P, E);
+    const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
+    const int64_t tok_tiles = (P + tile_rows - 1) / tile_rows + E;
 
     // gate/up projection with the SwiGLU epilogue -> h [P, I]
     CUtensorMap tw, tx;
     if ((st = encode_codes_map(&tw, w13_codes, H, 2 * I, E, 64)) != MXFP4_OK) return st;
-    if ((st = encode_act_map(&tx, w.x_sorted, H, P, nt)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, w.x_sorted, H, P, tiling.nt)) != MXFP4_OK) return st;
     mx::GemmArgs a{};
     a.w_scales = w13_scales;
     a.offsets = w.offsets;
@@ -397,7 +400,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     a.n_valid_feat = static_cast<int>(I);
     a.row_w = nullptr;
     a.status = d->status;
-    if ((e = mx::launch_grouped_gemm(mx::EPI_SWIGLU, nt, tw, tx, a,
+    if ((e = mx::launch_grouped_gemm(mx::EPI_SWIGLU, tiling, tw, tx, a,
                                      gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
         return cuda_fail(e);
 
@@ -409,7 +412,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
 
     // down projection, routing weight applied in fp32 -> y_sorted fp32 [P, H]
     if ((st = encode_codes_map(&tw, w2_codes, I, H, E, 128)) != MXFP4_OK) return st;
-    if ((st = encode_act_map(&tx, w.h, I, P, nt)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, w.h, I, P, tiling.nt)) != MXFP4_OK) return st;
     a.w_scales = w2_scales;
     a.K = static_cast<int>(I);
     a.rows_w = static_cast<int>(H);
@@ -419,7 +422,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     a.out_ld = H;
     a.n_valid_feat = static_cast<int>(H);
     a.row_w = w.w_sorted;
-    if ((e = mx::launch_grouped_gemm(mx::EPI_WEIGHTED, nt, tw, tx, a,
+    if ((e = mx::launch_grouped_gemm(mx::EPI_WEIGHTED, tiling, tw, tx, a,
                                      gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
         return cuda_fail(e);
 

@@ -11,24 +11,29 @@
 // 4.40 performance upgrades for OpenAI GPT-OSS ...", sections "What MXFP4 Is"
 // and "Zero-Build Kernels from the Hub").
 //
+// Work tile: 128 weight rows (the MMA's M side) x TT token tiles of NT rows
+// (the N side).  The weights are dequantized once per 64-wide K stage and used
+// by TT MMAs, so TT = 2 halves the dequant work and the weight traffic per flop.
+//
 // Data flow (one persistent CTA per SM, 16 warps):
-//   warp 0        TMA producer: per tile, the block scales of its 128 weight
-//                 rows (bulk copy, double-buffered across tiles); per 64-wide K
-//                 stage, the packed codes of the 128 rows (32 B per row,
-//                 32B-swizzled) and the bf16 activation tile [NT x 64]
-//                 (128B-swizzled) -> smem ring.
-//   warps 4..11   two dequant warpgroups (alternate stages): each thread owns
-//                 one weight row; codes -> bf16 through a 256-entry shared LUT
-//                 (lane-replicated, conflict-free) times the block scale 2^(S-127)
-//                 (exact bf16 product), stored with tcgen05.st into TMEM: the
-//                 dequantized weights are the MMA's A operand and never touch
-//                 shared memory.
-//   warp 1        MMA issuer: tcgen05.mma kind::f16, M = 128 weight rows,
-//                 N = NT tokens, K = 16 per instruction, A from TMEM, B from
-//                 smem, D (fp32) in TMEM, double-buffered across tiles.
-//   warps 12..15  epilogue: tcgen05.ld of the accumulator, fused epilogue,
+//   warp 0        codes producer: per tile the block scales of its 128 rows
+//                 (bulk copy, double-buffered); per K stage the packed codes
+//                 (32 B per row, 32B-swizzled) -> a deep codes ring that the
+//                 dequant warps release as soon as they have read it.
+//   warp 2        activation producer: per K stage TT bf16 tiles [NT x 64]
+//                 (128B-swizzled, the UMMA K-major layout) -> activation ring,
+//                 released by the MMA.
+//   warps 4..11   two dequant warpgroups (alternate stages): one weight row per
+//                 thread; codes -> bf16 through a lane-replicated 256-entry
+//                 shared LUT times the block scale 2^(S-127) (exact bf16
+//                 product), stored with tcgen05.st into TMEM: the dequantized
+//                 weights are the MMA's A operand and never touch shared memory.
+//   warp 1        MMA issuer: tcgen05.mma kind::f16, M = 128, N = NT, K = 16,
+//                 A from TMEM, B from shared memory, D (fp32) in TMEM.
+//   warps 12..15  epilogue: tcgen05.ld of the accumulators, fused epilogue,
 //                 stores.
-// TMEM: columns [0, 2*NT) the two accumulators, [256, 512) eight A slots.
+// TMEM: columns [0, 256) accumulators (TT*NT columns per buffer, double-buffered
+// when they fit), [256, 512) eight 32-column A slots.
 // Every mbarrier wait is time-bounded (MXFP4_ERR_TIMEOUT in the status word).
 #include "common.cuh"
 #include "internal.h"
@@ -42,40 +47,66 @@ constexpr int kBM = 128;            // weight rows per tile (MMA M)
 constexpr int kBK = 64;             // K per pipeline stage
 constexpr int kASlots = 8;          // TMEM A-operand slots (32 columns each)
 constexpr int kACol0 = 256;         // first TMEM column of the A slots
-constexpr int kCodeBytes = kBM * kBK / 2;
+constexpr int kSub = 4;             // 64-wide K sub-stages per codes super-stage
+constexpr int kCodeRowBytes = kSub * kBK / 2;          // 128 B of codes per weight row
+constexpr int kCodeBytes = kBM * kCodeRowBytes;        // one codes super-stage (16 KB)
 constexpr int kLutBytes = 256 * 256;
 constexpr int kMaxGroups = 256;
-constexpr int kXbufBytes = 2 * 2 * 32 * 16 * 4;
+constexpr int kXbufBytes = 0;
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kMaxRing = 16;
+constexpr int kMaxCodeStages = 4;
 
-template <int NT>
+template <int NT, int TT>
 struct Cfg {
-    static constexpr int kActBytes = NT * kBK * 2;
-    static constexpr int kStageBytes = kCodeBytes + kActBytes;
-    static constexpr int kMaxStages = NT == 16 ? 16 : (NT == 32 ? 12 : (NT == 64 ? 8 : 5));
-    static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-B alignment");
-    static_assert(2 * NT <= kACol0, "accumulators overlap the A slots");
+    static constexpr int kActTile = NT * kBK * 2;          // one token tile of one K stage
+    static constexpr int kActStage = TT * kActTile;
+    static constexpr int kAccCols = TT * NT;               // TMEM columns of one accumulator set
+    static constexpr int kAccBufs = 2 * kAccCols <= kACol0 ? 2 : 1;
+    static constexpr int kTileRows = TT * NT;               // token rows of a work tile
+    // NT <= 64: the activation ring has one stage per A slot and both are released by
+    // the same MMA commit (one commit per K stage instead of two).
+    static constexpr bool kLock = NT <= 64;
+    static constexpr int kMaxActStages = kLock ? kASlots : (TT == 1 ? 5 : 3);
+    static constexpr int kChunk = kAccCols < 32 ? kAccCols : 32;   // epilogue columns per TMEM load
+    static_assert(kActTile % 1024 == 0, "activation tiles must keep 1024-B alignment");
+    static_assert(kAccCols <= kACol0, "accumulators overlap the A slots");
 };
 
 // Shared-memory layout, identical on host (sizing) and device.
 struct Layout {
-    int stages_off, scales_off, scale_bytes, xbuf_off, bar_off, tstart_off, off_off, misc_off, total;
+    int codes_off, acts_off, scales_off, scale_bytes, xbuf_off, bar_off, tstart_off, off_off,
+        misc_off, total;
 };
 
-__host__ __device__ inline Layout make_layout(int stage_bytes, int stages, int K) {
+__host__ __device__ inline Layout make_layout(int act_stage_bytes, int code_stages, int act_stages,
+                                              int K) {
     Layout L;
-    L.stages_off = kLutBytes;
-    L.scales_off = L.stages_off + stages * stage_bytes;
+    L.codes_off = kLutBytes;
+    L.acts_off = L.codes_off + code_stages * kCodeBytes;
+    L.scales_off = L.acts_off + act_stages * act_stage_bytes;
     L.scale_bytes = ((kBM * (K / 32)) + 127) / 128 * 128;
     L.xbuf_off = L.scales_off + 2 * L.scale_bytes;
     L.bar_off = L.xbuf_off + kXbufBytes;
-    const int n_bars = 2 * 16 + 2 * kASlots + 4 + 4 + 1;
+    const int n_bars = 4 * kMaxRing + 2 * kASlots + 2 + 2 + 2 + 2 + 1;
     L.tstart_off = L.bar_off + n_bars * 8;
     L.off_off = L.tstart_off + (kMaxGroups + 1) * 4;
     L.misc_off = L.off_off + (kMaxGroups + 1) * 4;
     L.total = L.misc_off + 16 + 1024;   // + slack for the 1024-B alignment of the base
     return L;
 }
+
+// Position in a ring of n slots with the parity of the slot's current use.
+struct Ring {
+    int idx = 0;
+    uint32_t ph = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++idx == n) {
+            idx = 0;
+            ph ^= 1u;
+        }
+    }
+};
 
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -138,32 +169,6 @@ __device__ __forceinline__ void store_bf16(void* out, int64_t idx, float v) {
     reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
-struct TileInfo {
-    int g, f, row0, mrows;
-};
-
-// Tile t -> (group, feature tile, first row, valid rows).  Tiles of a group are
-// numbered feature-tile-major with the token tile fastest, so CTAs working at
-// the same time share the weight tile (L2 reuse).
-template <int NT>
-__device__ __forceinline__ TileInfo decode_tile(int t, const int* s_tstart, const int* s_off, int G) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {                 // largest g with s_tstart[g] <= t
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_tstart[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    TileInfo ti;
-    ti.g = lo;
-    const int m = s_off[lo + 1] - s_off[lo];
-    const int mt = (m + NT - 1) / NT;
-    const int local = t - s_tstart[lo];
-    ti.f = local / mt;
-    const int tt = local - ti.f * mt;
-    ti.row0 = s_off[lo] + tt * NT;
-    ti.mrows = min(NT, m - tt * NT);
-    return ti;
-}
-
 // Copy `rows` consecutive rows of block scales (kb bytes each) from global to
 // shared: the 16-byte multiple with one bulk copy (counted on `bar`), the tail
 // with plain loads.  Returns the bulk byte count.
@@ -180,29 +185,65 @@ __device__ __forceinline__ uint32_t stage_scales(uint8_t* dst, const uint8_t* sr
     return bulk;
 }
 
-template <int NT, int MODE>
+struct TileInfo {
+    int g, f, row0, mrows;
+};
+
+// The ki-th 64-wide K stage of a tile when its super-stages are visited starting at
+// super-stage `rot` (the last super-stage may hold fewer than kSub stages).
+__device__ __forceinline__ int stage_at(int ki, int rot, int nss, int nk) {
+    const int rot_stage = rot * kSub;              // stages visited before wrapping
+    const int first = nk - rot_stage;              // stages from super-stage rot to the end
+    return ki < first ? rot_stage + ki : ki - first;
+}
+
+// Work tile t -> (group, feature tile, first row, valid rows).  Tiles of a group
+// are numbered feature-tile-major with the token tile fastest, so CTAs working at
+// the same time share the weight tile (L2 reuse).
+__device__ __forceinline__ TileInfo decode_tile(int t, const int* s_tstart, const int* s_off, int G,
+                                                int tile_rows) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {                 // largest g with s_tstart[g] <= t
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_tstart[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    TileInfo ti;
+    ti.g = lo;
+    const int m = s_off[lo + 1] - s_off[lo];
+    const int mt = (m + tile_rows - 1) / tile_rows;
+    const int local = t - s_tstart[lo];
+    ti.f = local / mt;
+    const int tt = local - ti.f * mt;
+    ti.row0 = s_off[lo] + tt * tile_rows;
+    ti.mrows = min(tile_rows, m - tt * tile_rows);
+    return ti;
+}
+
+template <int NT, int TT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
-    using C = Cfg<NT>;
-    const int S_ = args.stages;
-    const Layout Ly = make_layout(C::kStageBytes, S_, args.K);
+    using C = Cfg<NT, TT>;
+    const int SC = args.code_stages, SA = args.act_stages;
+    const Layout Ly = make_layout(C::kActStage, SC, SA, args.K);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-    uint8_t* stages = smem + Ly.stages_off;
+    uint8_t* codes = smem + Ly.codes_off;
+    uint8_t* acts = smem + Ly.acts_off;
     uint8_t* scales = smem + Ly.scales_off;
-    float* xbuf = reinterpret_cast<float*>(smem + Ly.xbuf_off);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bar_off);
-    uint64_t* full = bars;                 // [16] stage filled (TMA tx)
-    uint64_t* empty = bars + 16;           // [16] stage consumed (MMA commit)
-    uint64_t* afull = bars + 32;           // [8]  A slot written (128 dequant threads)
-    uint64_t* aempty = afull + kASlots;    // [8]  A slot consumed (MMA commit)
-    uint64_t* accfull = aempty + kASlots;  // [2]  accumulator ready (MMA commit)
-    uint64_t* accempty = accfull + 2;      // [2]  accumulator drained (128 epilogue threads)
-    uint64_t* sfull = accempty + 2;        // [2]  tile scales staged (tx)
-    uint64_t* sempty = sfull + 2;          // [2]  tile scales no longer needed (MMA commit)
+    uint64_t* cfull = bars;                          // codes stage landed (TMA tx)
+    uint64_t* cempty = bars + kMaxRing;              // codes super-stage read (256 dequant threads)
+    uint64_t* xfull = bars + 2 * kMaxRing;           // activation stage landed (TMA tx)
+    uint64_t* xempty = bars + 3 * kMaxRing;          // activation stage consumed (MMA commit)
+    uint64_t* afull = bars + 4 * kMaxRing;           // A-slot set written (512 arrivals per group)
+    uint64_t* aempty = afull + kASlots;              // A-slot set consumed (MMA commit)
+    uint64_t* accfull = aempty + kASlots;            // accumulators ready (MMA commit)
+    uint64_t* accempty = accfull + 2;                // accumulators drained (128 epilogue threads)
+    uint64_t* sfull = accempty + 2;                  // tile scales staged (tx)
+    uint64_t* sempty = sfull + 2;                    // tile scales released (MMA commit)
     uint64_t* drain = sempty + 2;
     int* s_tstart = reinterpret_cast<int*>(smem + Ly.tstart_off);
     int* s_off = reinterpret_cast<int*>(smem + Ly.off_off);
@@ -213,15 +254,20 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = args.offsets ? args.G : 1;
     const int kb = args.K / 32;            // scale bytes per weight row
+    constexpr int NB = C::kAccBufs;
 
     // ---------------- set-up
     if (tid == 0) {
-        for (int s = 0; s < S_; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < SC; ++s) {
+            mbar_init(&cfull[s], 1);
+            mbar_init(&cempty[s], 256);   // both dequant warpgroups pass every super-stage
+        }
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], 1);
         }
         for (int a = 0; a < kASlots; ++a) {
-            mbar_init(&afull[a], 128);
+            mbar_init(&afull[a], 512);   // per group: 2 arrivals x 256 dequant threads
             mbar_init(&aempty[a], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -235,10 +281,8 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         *s_never = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tmap_w);
-        prefetch_tmap(&tmap_x);
-    }
+    if (warp == 0 && lane == 0) prefetch_tmap(&tmap_w);
+    if (warp == 2 && lane == 0) prefetch_tmap(&tmap_x);
     if (warp == 1) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
@@ -255,7 +299,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         for (int g = 0; g < G; ++g) {
             s_tstart[g] = acc;
             const int m = s_off[g + 1] - s_off[g];
-            acc += ((m + NT - 1) / NT) * args.n_ftiles;
+            acc += ((m + C::kTileRows - 1) / C::kTileRows) * args.n_ftiles;
         }
         s_tstart[G] = acc;
     }
@@ -264,16 +308,21 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const int total_tiles = s_tstart[G];
-    const int nk = args.K / kBK;
+    const int nk = args.K / kBK;                    // 64-wide K stages
+    const int nss = (nk + kSub - 1) / kSub;         // codes super-stages
+    // Every CTA walks the K super-stages of its tiles in a rotated order (starting at
+    // blockIdx.x mod nss): CTAs that share a token tile then read different activation
+    // lines at any moment instead of all hitting the same L2 lines together.
+    const int rot = static_cast<int>(blockIdx.x % static_cast<unsigned>(nss));
 
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- codes (+ scales) producer
         if (lane == 0) {
-            int kit = 0, lt = 0;
+            Ring c;
+            int lt = 0, issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
-                const TileInfo ti = decode_tile<NT>(t, s_tstart, s_off, G);
-                // block scales of the tile's weight rows, in the smem row order of the codes
+                const TileInfo ti = decode_tile(t, s_tstart, s_off, G, C::kTileRows);
                 const int sb = lt & 1;
                 if (!mbar_wait(&sempty[sb], ((lt >> 1) & 1) ^ 1, s_abort)) { ok = false; break; }
                 uint8_t* sdst = scales + sb * Ly.scale_bytes;
@@ -288,64 +337,146 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                     tx += stage_scales(sdst, gsc + static_cast<int64_t>(ti.f * kBM) * kb, rows, kb, &sfull[sb]);
                 }
                 mbar_arrive_expect_tx(&sfull[sb], tx);
-                for (int ks = 0; ks < nk; ++ks, ++kit) {
-                    const int st = kit % S_;
-                    const uint32_t ph = (kit / S_) & 1;
-                    if (!mbar_wait(&empty[st], ph ^ 1, s_abort)) { ok = false; break; }
-                    uint8_t* sb_ = stages + st * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+                // codes in super-stages of kSub K stages: 128 B of every weight row per
+                // TMA box (row segments this wide stream from HBM at full rate); the tail
+                // beyond K/2 bytes is zero-filled by the TMA and never dequantized
+                for (int si = 0; si < nss; ++si) {
+                    const int ss = si + rot < nss ? si + rot : si + rot - nss;
+                    if (!mbar_wait(&cempty[c.idx], c.ph ^ 1, s_abort)) { ok = false; break; }
+                    uint8_t* dst = codes + c.idx * kCodeBytes;
+                    mbar_arrive_expect_tx(&cfull[c.idx], kCodeBytes);
+                    const int x = ss * kCodeRowBytes;
                     if (MODE == EPI_SWIGLU) {
-                        tma_load_3d(sb_, &tmap_w, &full[st], ks * 32, ti.f * 64, ti.g);
-                        tma_load_3d(sb_ + 64 * 32, &tmap_w, &full[st], ks * 32, args.I + ti.f * 64, ti.g);
+                        tma_load_3d(dst, &tmap_w, &cfull[c.idx], x, ti.f * 64, ti.g);
+                        tma_load_3d(dst + 64 * kCodeRowBytes, &tmap_w, &cfull[c.idx], x, args.I + ti.f * 64, ti.g);
                     } else {
-                        tma_load_3d(sb_, &tmap_w, &full[st], ks * 32, ti.f * kBM, ti.g);
+                        tma_load_3d(dst, &tmap_w, &cfull[c.idx], x, ti.f * kBM, ti.g);
                     }
-                    tma_load_2d(sb_ + kCodeBytes, &tmap_x, &full[st], ks * kBK, ti.row0);
+                    c.next(SC);
+                    ++issued;
                 }
             }
             if (!ok) {
                 *s_abort = 1;
                 record_status(args.status, MXFP4_ERR_TIMEOUT);
                 // let the copies already issued land before the CTA exits
-                const int n_inflight = kit < S_ ? kit : S_;
-                for (int i = 1; i <= n_inflight; ++i) {
-                    const int k2 = kit - i;
-                    mbar_wait(&full[k2 % S_], (k2 / S_) & 1, s_never);
+                Ring r;
+                const int first = issued > SC ? issued - SC : 0;
+                for (int i = 0; i < issued; ++i) {
+                    if (i >= first) mbar_wait(&cfull[r.idx], r.ph, s_never);
+                    r.next(SC);
                 }
-                for (int i = 1; i <= 2 && i <= lt + 1; ++i) {
-                    const int l2 = lt + 1 - i;
+                for (int l2 = lt - 1; l2 <= lt && l2 >= 0; ++l2)
                     mbar_wait(&sfull[l2 & 1], (l2 >> 1) & 1, s_never);
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------- activation producer
+        if (lane == 0) {
+            Ring x;             // kLock: ring of A-slot sets (2); else: ring of stages (SA)
+            int issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                const TileInfo ti = decode_tile(t, s_tstart, s_off, G, C::kTileRows);
+                for (int si = 0; si < nss && ok; ++si) {
+                    const int ss = si + rot < nss ? si + rot : si + rot - nss;
+                    const int nsub = min(kSub, nk - ss * kSub);
+                    if (C::kLock) {
+                        // one slot per stage of the group, released with the group's A slots
+                        if (!mbar_wait(&aempty[x.idx], x.ph ^ 1, s_abort)) { ok = false; break; }
+                        for (int j = 0; j < kSub; ++j) {
+                            const int slot = x.idx * kSub + j;
+                            if (j < nsub) {
+                                mbar_arrive_expect_tx(&xfull[slot], C::kActStage);
+#pragma unroll
+                                for (int tt = 0; tt < TT; ++tt)
+                                    tma_load_2d(acts + slot * C::kActStage + tt * C::kActTile, &tmap_x, &xfull[slot],
+                                                (ss * kSub + j) * kBK, ti.row0 + tt * NT);
+                            } else {
+                                mbar_arrive(&xfull[slot]);   // unused slot of a short group: keep phases aligned
+                            }
+                        }
+                        x.next(2);
+                        ++issued;
+                    } else {
+                        for (int j = 0; j < nsub; ++j) {
+                            if (!mbar_wait(&xempty[x.idx], x.ph ^ 1, s_abort)) { ok = false; break; }
+                            mbar_arrive_expect_tx(&xfull[x.idx], C::kActStage);
+#pragma unroll
+                            for (int tt = 0; tt < TT; ++tt)
+                                tma_load_2d(acts + x.idx * C::kActStage + tt * C::kActTile, &tmap_x, &xfull[x.idx],
+                                            (ss * kSub + j) * kBK, ti.row0 + tt * NT);
+                            x.next(SA);
+                            ++issued;
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                *s_abort = 1;
+                record_status(args.status, MXFP4_ERR_TIMEOUT);
+                // let the copies already issued land before the CTA exits
+                if (C::kLock) {
+                    Ring r;
+                    const int first = issued > 2 ? issued - 2 : 0;
+                    for (int i = 0; i < issued; ++i) {
+                        if (i >= first)
+                            for (int j = 0; j < kSub; ++j) mbar_wait(&xfull[r.idx * kSub + j], r.ph, s_never);
+                        r.next(2);
+                    }
+                } else {
+                    Ring r;
+                    const int first = issued > SA ? issued - SA : 0;
+                    for (int i = 0; i < issued; ++i) {
+                        if (i >= first) mbar_wait(&xfull[r.idx], r.ph, s_never);
+                        r.next(SA);
+                    }
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer
+        // One barrier wait and one commit per group of kSub K stages: a wait issued
+        // between tcgen05 operations stalls the issuing thread for roughly the latency
+        // of the MMAs in flight, so it is paid once per group, not once per stage.
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kBM, NT);
-            int kit = 0, lt = 0;
+            Ring x, a;          // x: activation stages (only when !kLock); a: A-slot sets
+            int lt = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
-                const int acc = lt & 1;
-                if (!mbar_wait(&accempty[acc], ((lt >> 1) & 1) ^ 1, s_abort)) { ok = false; break; }
+                const int b = NB == 2 ? (lt & 1) : 0;
+                const uint32_t bph = NB == 2 ? ((lt >> 1) & 1) : (lt & 1);
+                if (!mbar_wait(&accempty[b], bph ^ 1, s_abort)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * NT;
-                for (int ks = 0; ks < nk; ++ks, ++kit) {
-                    const int st = kit % S_;
-                    const int as = kit % kASlots;
-                    if (!mbar_wait(&full[st], (kit / S_) & 1, s_abort) ||
-                        !mbar_wait(&afull[as], (kit / kASlots) & 1, s_abort)) { ok = false; break; }
+                const uint32_t d_tmem = tmem_base + b * C::kAccCols;
+                int ki = 0;
+                for (int si = 0; si < nss; ++si) {
+                    const int ss = si + rot < nss ? si + rot : si + rot - nss;
+                    const int nsub = min(kSub, nk - ss * kSub);
+                    if (!mbar_wait(&afull[a.idx], a.ph, s_abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t b_base = smem_u32(stages + st * C::kStageBytes + kCodeBytes);
-                    const uint32_t a_tmem = tmem_base + kACol0 + as * 32;
+                    for (int j = 0; j < nsub; ++j, ++ki) {
+                        const int xs = C::kLock ? a.idx * kSub + j : x.idx;
+                        const uint32_t b_base = smem_u32(acts + xs * C::kActStage);
+                        const uint32_t a_tmem = tmem_base + kACol0 + (a.idx * kSub + j) * 32;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mma_bf16_ts(d_tmem, a_tmem + 8 * j, sw128_desc(b_base + 32 * j), idesc,
-                                    (ks | j) != 0 ? 1u : 0u);
-                    tc_commit(&empty[st]);
-                    tc_commit(&aempty[as]);
+                        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+                                mma_bf16_ts(d_tmem + tt * NT, a_tmem + 8 * jj,
+                                            sw128_desc(b_base + tt * C::kActTile + 32 * jj), idesc,
+                                            (ki | jj) != 0 ? 1u : 0u);
+                        if (!C::kLock) {
+                            tc_commit(&xempty[x.idx]);
+                            x.next(SA);
+                        }
+                    }
+                    tc_commit(&aempty[a.idx]);
+                    a.next(2);
                 }
                 if (!ok) break;
-                tc_commit(&accfull[acc]);
+                tc_commit(&accfull[b]);
                 tc_commit(&sempty[lt & 1]);
             }
             if (!ok) {
@@ -363,41 +494,61 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         const uint32_t lut_lane = smem_u32(lut) + lane * 4;
         int srow;
         if (MODE == EPI_SWIGLU) {
-            const int half = q >> 1, up = q & 1;
-            srow = up * 64 + half * 32 + lane;  // lanes: gate 0-31 | up 0-31 | gate 32-63 | up 32-63
+            // smem rows 0-63 gate, 64-127 up; lane l of warp q: feature 16q + (l & 15),
+            // gate for l < 16, up for l >= 16
+            srow = (lane < 16 ? 0 : 64) + 16 * q + (lane & 15);
         } else {
             srow = q * 32 + lane;
         }
-        const uint32_t sw = (static_cast<uint32_t>(srow) >> 2) & 1u;
+        const uint32_t sw = static_cast<uint32_t>(srow) & 7u;   // 128B swizzle: chunk ^= row % 8
+        const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
+        Ring c, a, xr;        // codes super-stages, A-slot sets, activation stages (!kLock)
         int kit = 0, lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
-            const TileInfo ti = decode_tile<NT>(t, s_tstart, s_off, G);
+            const TileInfo ti = decode_tile(t, s_tstart, s_off, G, C::kTileRows);
             const bool valid = MODE == EPI_SWIGLU || ti.f * kBM + srow < args.rows_w;
             const uint32_t sc_row = smem_u32(scales + (lt & 1) * Ly.scale_bytes) + srow * kb;
-            bool scales_ready = false;
-            for (int ks = 0; ks < nk; ++ks, ++kit) {
-                if ((kit & 1) != d) continue;
-                const int st = kit % S_;
-                const int as = kit % kASlots;
-                bool got = mbar_wait(&full[st], (kit / S_) & 1, s_abort) &&
-                           mbar_wait(&aempty[as], ((kit / kASlots) & 1) ^ 1, s_abort);
-                if (!scales_ready)
-                    got = got && mbar_wait(&sfull[lt & 1], (lt >> 1) & 1, s_abort);
+            for (int si = 0; si < nss && ok; ++si) {
+                const int ss = si + rot < nss ? si + rot : si + rot - nss;
+                const int nsub = min(kSub, nk - ss * kSub);
+                // the group's A slots are free, its codes have landed, the tile's scales too
+                bool got = mbar_wait(&aempty[a.idx], a.ph ^ 1, s_abort) &&
+                           mbar_wait(&cfull[c.idx], c.ph, s_abort);
+                if (si == 0) got = got && mbar_wait(&sfull[lt & 1], (lt >> 1) & 1, s_abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
-                scales_ready = true;
                 tc_fence_after();
-                const uint32_t sc = valid ? lds_u16(sc_row + 2 * ks) : 0x7F7Fu;
-                const uint32_t row_addr = smem_u32(stages + st * C::kStageBytes) + srow * 32;
-                const uint4 c0 = lds128(row_addr + ((0u ^ sw) << 4));
-                const uint4 c1 = lds128(row_addr + ((1u ^ sw) << 4));
-                uint32_t out[32];
-                dequant_block16(c0, sc & 0xFFu, lut_lane, out);
-                dequant_block16(c1, sc >> 8, lut_lane, out + 16);
-                tmem_st_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + as * 32, out);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&afull[as]);
+                const uint32_t row_addr = smem_u32(codes + c.idx * kCodeBytes) + srow * kCodeRowBytes;
+                int done = 0;
+                for (int j = 0; j < nsub; ++j, ++kit) {
+                    const int xs = C::kLock ? a.idx * kSub + j : xr.idx;
+                    const uint32_t xph = C::kLock ? a.ph : xr.ph;
+                    if ((kit & 1) == d) {
+                        const int ks = ss * kSub + j;
+                        const uint32_t sc = valid ? lds_u16(sc_row + 2 * ks) : 0x7F7Fu;
+                        const uint4 c0 = lds128(row_addr + (((2u * j) ^ sw) << 4));
+                        const uint4 c1 = lds128(row_addr + (((2u * j + 1u) ^ sw) << 4));
+                        uint32_t out[32];
+                        dequant_block16(c0, sc & 0xFFu, lut_lane, out);
+                        dequant_block16(c1, sc >> 8, lut_lane, out + 16);
+                        tmem_st_x32(tmem_lane + (a.idx * kSub + j) * 32, out);
+                        tmem_wait_st();
+                        // the stage's activation tile must have landed too: the MMA issuer
+                        // waits on the group barrier only
+                        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&xfull[xs], xph, s_abort))) { ok = false; break; }
+                        tc_fence_before();
+                        mbar_arrive(&afull[a.idx]);
+                        ++done;
+                    }
+                    if (!C::kLock) xr.next(SA);
+                }
+                if (!ok) break;
+                // every dequant thread arrives exactly twice per group (a group has four
+                // stages, two per warpgroup); short groups are topped up here
+                for (; done < 2; ++done) mbar_arrive(&afull[a.idx]);
+                mbar_arrive(&cempty[c.idx]);     // this warpgroup is done with the super-stage
+                c.next(SC);
+                a.next(2);
             }
         }
         if (!ok) {
@@ -406,49 +557,45 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         }
     } else if (warp >= 12) {
         // ---------------- epilogue warpgroup
+        constexpr int CW = C::kChunk;
+        constexpr int NCH = C::kAccCols / CW;
         const int q = warp & 3;
-        int lt = 0, cc = 0;
+        const bool lo = lane < 16;
+        int lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
-            const TileInfo ti = decode_tile<NT>(t, s_tstart, s_off, G);
-            const int acc = lt & 1;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&accfull[acc], (lt >> 1) & 1, s_abort))) { ok = false; break; }
+            const TileInfo ti = decode_tile(t, s_tstart, s_off, G, C::kTileRows);
+            const int b = NB == 2 ? (lt & 1) : 0;
+            const uint32_t bph = NB == 2 ? ((lt >> 1) & 1) : (lt & 1);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&accfull[b], bph, s_abort))) { ok = false; break; }
             tc_fence_after();
-            const uint32_t t_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NT;
-#pragma unroll 1
-            for (int c = 0; c < NT / 16; ++c, ++cc) {
-                uint32_t v[16];
-                tmem_ld_x16(t_base + 16 * c, v);
-                tmem_wait_ld();
+            const uint32_t t_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::kAccCols;
+            // column j of the accumulator set is token row ti.row0 + j
+            auto process = [&](const uint32_t* cur, int c) {
                 if (MODE == EPI_SWIGLU) {
-                    const int pr = q >> 1, up = q & 1;
-                    // [pair][buffer][n][lane]: lanes write consecutive words (no bank conflicts)
-                    float* xb = xbuf + (pr * 2 + (cc & 1)) * 16 * 32 + lane;
-                    if (!up) {
+                    // lanes < 16 finish columns [0, CW/2) of the chunk, lanes >= 16 columns
+                    // [CW/2, CW); each needs its partner's (lane ^ 16) gate or up value
+                    const int feat = ti.f * 64 + 16 * q + (lane & 15);
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) xb[n * 32] = __uint_as_float(v[n]);
-                    }
-                    named_bar_sync(1 + pr, 64);
-                    if (up) {
-                        const int feat = ti.f * 64 + pr * 32 + lane;
-#pragma unroll
-                        for (int n = 0; n < 16; ++n) {
-                            const int tok = 16 * c + n;
-                            if (tok < ti.mrows) {
-                                const float h = silu_f32(xb[n * 32]) * __uint_as_float(v[n]);
-                                store_bf16(args.out, static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat, h);
-                            }
-                        }
+                    for (int i = 0; i < CW / 2; ++i) {
+                        const uint32_t send = lo ? cur[CW / 2 + i] : cur[i];
+                        const float other = __uint_as_float(__shfl_xor_sync(0xFFFFFFFFu, send, 16));
+                        const float g = lo ? __uint_as_float(cur[i]) : other;
+                        const float u = lo ? other : __uint_as_float(cur[CW / 2 + i]);
+                        const int tok = c * CW + (lo ? i : CW / 2 + i);
+                        if (tok < ti.mrows)
+                            store_bf16(args.out, static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat,
+                                       silu_f32(g) * u);
                     }
                 } else {
                     const int feat = ti.f * kBM + q * 32 + lane;
                     if (feat < args.n_valid_feat) {
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) {
-                            const int tok = 16 * c + n;
+                        for (int n = 0; n < CW; ++n) {
+                            const int tok = c * CW + n;
                             if (tok < ti.mrows) {
                                 const int64_t idx = static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat;
-                                const float val = __uint_as_float(v[n]);
+                                const float val = __uint_as_float(cur[n]);
                                 if (MODE == EPI_WEIGHTED)   // fp32 out: one rounding, in the combine
                                     reinterpret_cast<float*>(args.out)[idx] = val * args.row_w[ti.row0 + tok];
                                 else
@@ -457,9 +604,26 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         }
                     }
                 }
+            };
+            auto load = [&](uint32_t* dst, int c) {
+                if (CW == 32) tmem_ld_x32(t_base + c * CW, dst); else tmem_ld_x16(t_base + c * CW, dst);
+            };
+            // two register buffers: the next chunk's TMEM load overlaps this chunk's work
+            uint32_t v0[CW], v1[CW];
+            load(v0, 0);
+#pragma unroll 1
+            for (int c = 0; c < NCH; c += 2) {
+                tmem_wait_ld();
+                if (c + 1 < NCH) load(v1, c + 1);
+                process(v0, c);
+                if (c + 1 < NCH) {
+                    tmem_wait_ld();
+                    if (c + 2 < NCH) load(v0, c + 2);
+                    process(v1, c + 1);
+                }
             }
             tc_fence_before();
-            mbar_arrive(&accempty[acc]);
+            mbar_arrive(&accempty[b]);
         }
         if (!ok) {
             *s_abort = 1;
@@ -475,62 +639,87 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     }
 }
 
-template <int NT, int MODE>
-cudaError_t launch_nt(const CUtensorMap& tw, const CUtensorMap& tx, GemmArgs a, int grid,
-                      cudaStream_t stream) {
-    using C = Cfg<NT>;
-    // deepest ring that fits next to the LUT, the scale buffers and the rest
-    int stages = C::kMaxStages;
-    while (stages > 2 && make_layout(C::kStageBytes, stages, a.K).total > kSmemLimit) --stages;
-    const Layout L = make_layout(C::kStageBytes, stages, a.K);
-    if (stages < 3 || L.total > kSmemLimit) return cudaErrorInvalidConfiguration;
-    a.stages = stages;
-    auto kern = grouped_w4a16_kernel<NT, MODE>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+// Ring depths for a launch: the deepest rings that fit next to the LUT, the
+// scale buffers and the rest (activation ring first, then the codes ring).
+template <int NT, int TT>
+bool ring_depths(int K, int* sc, int* sa, int* smem) {
+    using C = Cfg<NT, TT>;
+    // The activation ring must hold at least one whole group of kSub stages: the MMA
+    // issuer consumes a group only once all its stages are ready.
+    int c = kMaxCodeStages, a = C::kMaxActStages;
+    while (make_layout(C::kActStage, c, a, K).total > kSmemLimit) {
+        if (c > 2) --c;
+        else if (!C::kLock && a > kSub) --a;
+        else return false;
+    }
+    *sc = c;
+    *sa = a;
+    *smem = make_layout(C::kActStage, c, a, K).total;
+    return true;
+}
+
+template <int NT, int TT, int MODE>
+cudaError_t launch_cfg(const CUtensorMap& tw, const CUtensorMap& tx, GemmArgs a, int grid,
+                       cudaStream_t stream) {
+    int sc = 0, sa = 0, smem = 0;
+    if (!ring_depths<NT, TT>(a.K, &sc, &sa, &smem)) return cudaErrorInvalidConfiguration;
+    a.code_stages = sc;
+    a.act_stages = sa;
+    auto kern = grouped_w4a16_kernel<NT, TT, MODE>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, L.total, stream>>>(tw, tx, a);
+    kern<<<grid, kThreads, smem, stream>>>(tw, tx, a);
     return cudaGetLastError();
 }
 
 template <int MODE>
-cudaError_t launch_mode(int nt, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
-                        int grid, cudaStream_t stream) {
-    switch (nt) {
-        case 16: return launch_nt<16, MODE>(tw, tx, a, grid, stream);
-        case 32: return launch_nt<32, MODE>(tw, tx, a, grid, stream);
-        case 64: return launch_nt<64, MODE>(tw, tx, a, grid, stream);
-        default: return launch_nt<128, MODE>(tw, tx, a, grid, stream);
-    }
+cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap& tx,
+                        const GemmArgs& a, int grid, cudaStream_t stream) {
+    if (nt == 16) return launch_cfg<16, 1, MODE>(tw, tx, a, grid, stream);
+    if (nt == 32) return launch_cfg<32, 1, MODE>(tw, tx, a, grid, stream);
+    if (nt == 64) return launch_cfg<64, 1, MODE>(tw, tx, a, grid, stream);
+    (void)tt;
+    return launch_cfg<128, 1, MODE>(tw, tx, a, grid, stream);
 }
 
 }  // namespace
 
-int pick_token_tile(int64_t rows, int64_t groups) {
+// Token tiling for `rows` activation rows spread over `groups` groups: NT rows per
+// MMA (16..128) and TT token tiles per dequantized weight tile.
+TokenTiling pick_token_tiling(int64_t rows, int64_t groups) {
     const int64_t avg = (rows + groups - 1) / (groups > 0 ? groups : 1);
-    if (avg <= 16) return 16;
-    if (avg <= 32) return 32;
-    if (avg <= 64) return 64;
-    return 128;
+    if (avg <= 16) return {16, 1};
+    if (avg <= 32) return {32, 1};
+    if (avg <= 64) return {64, 1};
+    return {128, 1};
 }
 
-// Largest K the kernel accepts (its tile's block scales must fit in shared memory
-// next to a 3-stage ring at the largest token tile).
+// Largest K the kernel accepts: a tile's block scales must fit in shared memory
+// next to the smallest rings of every configuration.
 int64_t max_gemm_k() {
     int64_t k = 64;
-    while (make_layout(Cfg<128>::kStageBytes, 3, static_cast<int>(k + 64)).total <= kSmemLimit) k += 64;
+    int sc, sa, smem;
+    while (ring_depths<128, 1>(static_cast<int>(k + 64), &sc, &sa, &smem) &&
+           ring_depths<64, 1>(static_cast<int>(k + 64), &sc, &sa, &smem) &&
+           ring_depths<32, 1>(static_cast<int>(k + 64), &sc, &sa, &smem) &&
+           ring_depths<16, 1>(static_cast<int>(k + 64), &sc, &sa, &smem))
+        k += 64;
     return k;
 }
 
 // Host launcher.  `tmap_w` covers the codes as a 3-D tensor {K/2, rows_w, G}
 // with box {32, 64 (SWIGLU) or 128, 1} and 32B swizzle; `tmap_x` covers the
 // activations {K, rows} (bf16) with box {64, nt} and 128B swizzle.
-cudaError_t launch_grouped_gemm(int mode, int nt, const CUtensorMap& tmap_w,
+cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream) {
     switch (mode) {
-        case EPI_SWIGLU: return launch_mode<EPI_SWIGLU>(nt, tmap_w, tmap_x, args, grid, stream);
-        case EPI_WEIGHTED: return launch_mode<EPI_WEIGHTED>(nt, tmap_w, tmap_x, args, grid, stream);
-        default: return launch_mode<EPI_PLAIN>(nt, tmap_w, tmap_x, args, grid, stream);
+        case EPI_SWIGLU:
+            return launch_mode<EPI_SWIGLU>(tiling.nt, tiling.tt, tmap_w, tmap_x, args, grid, stream);
+        case EPI_WEIGHTED:
+            return launch_mode<EPI_WEIGHTED>(tiling.nt, tiling.tt, tmap_w, tmap_x, args, grid, stream);
+        default:
+            return launch_mode<EPI_PLAIN>(tiling.nt, tiling.tt, tmap_w, tmap_x, args, grid, stream);
     }
 }
 

@@ -25,7 +25,15 @@ struct GemmArgs {
     int n_valid_feat;          // valid output columns
     const float* row_w;        // WEIGHTED: per-row scalar
     unsigned* status;          // device status word
-    int stages;                // smem pipeline depth (set by launch_grouped_gemm)
+    int code_stages;           // ring depths (set by launch_grouped_gemm)
+    int act_stages;
+};
+
+// Token tiling of the grouped GEMM: NT token rows per MMA, TT token tiles per
+// dequantized weight tile.
+struct TokenTiling {
+    int nt;
+    int tt;
 };
 
 cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t cols,
@@ -42,9 +50,9 @@ cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, i
                          void* x_sorted, int sm_count, cudaStream_t stream);
 cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, int top_k,
                            int64_t H, void* out, int sm_count, cudaStream_t stream);
-int pick_token_tile(int64_t rows, int64_t groups);
+TokenTiling pick_token_tiling(int64_t rows, int64_t groups);
 int64_t max_gemm_k();   // largest contraction length the grouped GEMM accepts
-cudaError_t launch_grouped_gemm(int mode, int nt, const CUtensorMap& tmap_w,
+cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream);
 
