@@ -140,6 +140,33 @@ MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,
 MXFP4_API size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k,
                                 mxfp4_mode mode);
 
+/* ---------------------------------------------------------------- allocation-free MoE layer
+ * Not a step of the method: the pages have no counterpart of this entry point.
+ *
+ * The same layer as moe_mxfp4_mlp, for callers that cannot allocate a workspace:
+ * cudaMalloc / cudaFree synchronize the whole device and can fail under memory
+ * pressure, so latency-critical decode loops, plugin hosts that hand out no device
+ * allocator, and code whose memory budget is owned by another framework must not
+ * allocate per call.  This entry point takes no workspace and allocates nothing; its
+ * scratch is one fixed array of MXFP4_NOALLOC_SCRATCH_BYTES in device memory, set
+ * aside on every GPU that loads the library until the process exits.
+ *   - Limit: calls whose moe_mxfp4_workspace_size(...) exceeds
+ *     MXFP4_NOALLOC_SCRATCH_BYTES return MXFP4_ERR_WORKSPACE (with H = I = 2880 and
+ *     32 experts that is up to 724 token-expert pairs, T * top_k: decode batches).
+ *   - The first call on each device looks up the array's device address (a host-side
+ *     query, no allocation); make that first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other streams, or
+ *     other host threads) race on it and must be serialized by the caller.  Nothing
+ *     carries over between calls: each call writes every scratch byte it reads.
+ * Arguments, layouts, results and the other errors are those of moe_mxfp4_mlp. */
+#define MXFP4_NOALLOC_SCRATCH_BYTES (16u << 20)
+MXFP4_API mxfp4_status moe_mxfp4_mlp_noalloc(const void* x_bf16, int64_t T, int64_t H,
+                                             const float* router_logits, int64_t E, int32_t top_k,
+                                             const uint8_t* w13_codes, const uint8_t* w13_scales,
+                                             int64_t I, const uint8_t* w2_codes,
+                                             const uint8_t* w2_scales, void* out_bf16,
+                                             mxfp4_mode mode, void* stream);
+
 /* ---------------------------------------------------------------- tracing
  * Optional stage timing for the calling host thread.  `events` points to
  * `n_events` cudaEvent_t handles (passed as void*) created by the caller; while

@@ -24,7 +24,8 @@ from ._lib import (Mxfp4Error, Mxfp4LibraryMissing, SCALE_CEIL, SCALE_FLOOR, W4A
 __all__ = [
     "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_gemm_workspace_size",
     "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
-    "moe_mxfp4_workspace_size", "mxfp4_get_device_status", "mxfp4_set_trace_events",
+    "moe_mxfp4_workspace_size", "moe_mxfp4_mlp_noalloc", "mxfp4_get_device_status",
+    "mxfp4_set_trace_events",
     "Mxfp4Error", "Mxfp4LibraryMissing",
     "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
 ]
@@ -146,6 +147,24 @@ def moe_mxfp4_mlp(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13_codes, 
         _p(x), T, H, _p(logits), E, top_k, _p(w13_codes), _p(w13_scales), I, _p(w2_codes),
         _p(w2_scales), _p(out), int(mode), _p(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+    return out
+
+
+def moe_mxfp4_mlp_noalloc(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13_codes, w13_scales,
+                          w2_codes, w2_scales, mode: int = W4A16, out=None, stream=None):
+    """The MoE layer of ``moe_mxfp4_mlp`` without a workspace, for callers that must not
+    allocate device memory per call (cudaMalloc synchronizes the device and can fail
+    under memory pressure).  Its scratch is a fixed 16 MiB array inside the library,
+    shared by all calls: calls that overlap on the GPU race on it.  ``out`` is the
+    caller's; pass it to keep this call allocation-free on the Python side too."""
+    lib = _lib.load()
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w13_codes.shape[1] // 2
+    out = _empty((T, H), torch.bfloat16, x) if out is None else out
+    _lib.check("moe_mxfp4_mlp_noalloc", lib.moe_mxfp4_mlp_noalloc(
+        _p(x), T, H, _p(logits), E, top_k, _p(w13_codes), _p(w13_scales), I, _p(w2_codes),
+        _p(w2_scales), _p(out), int(mode), _stream(stream)))
     return out
 
 

@@ -26,6 +26,7 @@ ERR_CUDA = 6
 ERR_TIMEOUT = 7
 
 IN_BF16, IN_F32 = 0, 1
+NOALLOC_SCRATCH_BYTES = 16 << 20   # MXFP4_NOALLOC_SCRATCH_BYTES in include/mxfp4.h
 SCALE_FLOOR, SCALE_CEIL = 0, 1
 W4A16, W4A4 = 0, 1
 
@@ -55,6 +56,8 @@ _SIGS = {
     "moe_mxfp4_mlp": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
                                      ctypes.c_int, _vp, _sz, _vp]),
     "moe_mxfp4_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, ctypes.c_int]),
+    "moe_mxfp4_mlp_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
+                                             ctypes.c_int, _vp]),
     "mxfp4_get_device_status": (ctypes.c_int, [_vp]),
     "mxfp4_set_trace_events": (None, [_vp, ctypes.c_int]),
     "mxfp4_last_cuda_error": (ctypes.c_int, []),

@@ -435,4 +435,53 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     return MXFP4_OK;
 }
 
+// ---------------------------------------------------------------- allocation-free MoE layer
+// Scratch of moe_mxfp4_mlp_noalloc: a fixed array in device memory, set aside on every
+// GPU that loads this library until the process exits.  Host code may not use the
+// array's name as a device address; the address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_moe_noalloc_scratch[MXFP4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (queried on first use).
+mxfp4_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return MXFP4_ERR_ARCH;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_moe_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return MXFP4_OK;
+}
+}  // namespace
+
+mxfp4_status moe_mxfp4_mlp_noalloc(const void* x_bf16, int64_t T, int64_t H,
+                                   const float* router_logits, int64_t E, int32_t top_k,
+                                   const uint8_t* w13_codes, const uint8_t* w13_scales, int64_t I,
+                                   const uint8_t* w2_codes, const uint8_t* w2_scales,
+                                   void* out_bf16, mxfp4_mode mode, void* stream) {
+    mxfp4_status st = check_route_args(router_logits, T, E, top_k);
+    if (st != MXFP4_OK) return st;
+    if (H <= 0 || I <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (moe_mxfp4_workspace_size(T, H, I, E, top_k, mode) > MXFP4_NOALLOC_SCRATCH_BYTES)
+        return MXFP4_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((st = device_info(&d)) != MXFP4_OK) return st;
+    void* ws = nullptr;
+    if ((st = noalloc_scratch(&ws)) != MXFP4_OK) return st;
+    // every scratch byte the layer reads is written earlier in the same call, so the
+    // previous call's leftovers need no clearing
+    return moe_mxfp4_mlp(x_bf16, T, H, router_logits, E, top_k, w13_codes, w13_scales, I,
+                         w2_codes, w2_scales, out_bf16, mode, ws, MXFP4_NOALLOC_SCRATCH_BYTES,
+                         stream);
+}
+
 }  // extern "C"
