@@ -38,7 +38,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 METRIC = "MXFP4 MoE GEMM TFLOP/s & weight GB/s vs roofline; quantize GB/s (1 B200)"
-L2_FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20          # B200 L2
 KERNELS_PER_LAYER = {0: 6, 1: 8}   # W4A16: route x3, gate/up, down, combine; W4A4: + 2 quantize
 
 
@@ -170,18 +170,18 @@ def make_events(n):
     return evs
 
 
-def time_layer(L, cfg, mode, steps, warmup, dev, world=1, trace=True, flush=None):
-    """Device time of `steps` layer calls (inputs resident), L2 flushed before each.
-    Returns per-step ms, per-stage ms (gate/up, down, ...) and the outer wall."""
+def time_layer(L, cfg, mode, steps, warmup, dev, world=1, trace=True):
+    """Device time of `steps` back-to-back layer calls (inputs resident).  No L2 flush:
+    every call streams all expert weights (>= 423 MB, over 3x the L2), so a step
+    finds at most the tail of the previous step's weights in L2.  Returns per-step ms,
+    per-stage ms (gate/up, down, ...) and the outer wall."""
     import moe_expert_gemm_mxfp4_b200 as mx
     T = L["x"].shape[0]
     xd, ld = L["x"].to(dev), L["logits"].to(dev)
     out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
     ws = torch.empty((mx.moe_mxfp4_workspace_size(T, cfg.H, cfg.I, cfg.E, cfg.top_k, mode),),
                      dtype=torch.uint8, device=dev)
-    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev) if flush is None else flush
     for _ in range(warmup):
-        flush.zero_()
         mx.moe_mxfp4_mlp(xd, ld, cfg.top_k, *L["w"], mode=mode, out=out, ws=ws)
     torch.cuda.synchronize()
     assert mx.mxfp4_get_device_status() == 0
@@ -192,7 +192,6 @@ def time_layer(L, cfg, mode, steps, warmup, dev, world=1, trace=True, flush=None
     torch.cuda.synchronize()
     outer0.record()
     for i in range(steps):
-        flush.zero_()
         if trace:
             mx.mxfp4_set_trace_events(stage[i])
         starts[i].record()
@@ -244,16 +243,16 @@ def time_e2e(L, cfg, mode, steps, warmup, dev):
     return a.elapsed_time(b) / steps, hx.numel() * 2 + hl.numel() * 4, hout.numel() * 2
 
 
-def time_kernel(fn, steps, warmup, dev, flush):
-    for _ in range(warmup):
-        flush.zero_()
-        fn()
+def time_kernel(fn, steps, warmup, dev):
+    """Mean device time of fn(i), i = 0..steps-1; fn rotates over enough buffers that
+    one call finds none of its data in L2."""
+    for i in range(warmup):
+        fn(i)
     torch.cuda.synchronize()
     s, e = make_events(steps), make_events(steps)
     for i in range(steps):
-        flush.zero_()
         s[i].record()
-        fn()
+        fn(i)
         e[i].record()
     torch.cuda.synchronize()
     return statistics.mean(a.elapsed_time(b) for a, b in zip(s, e))
@@ -261,7 +260,7 @@ def time_kernel(fn, steps, warmup, dev, flush):
 
 # ------------------------------------------------------------------ breakdown lines
 
-def bench_quant(dev, pk, flush, steps=20, warmup=5):
+def bench_quant(dev, pk, steps=20, warmup=5):
     import moe_expert_gemm_mxfp4_b200 as mx
     from moe_expert_gemm_mxfp4_b200 import inputs
     x = inputs.quant_tensor().to(dev)
@@ -270,8 +269,16 @@ def bench_quant(dev, pk, flush, steps=20, warmup=5):
     scales = torch.empty((R, C // 32), dtype=torch.uint8, device=dev)
     out = torch.empty_like(x)
     nbytes = R * C * 2 + R * C // 2 + R * C // 32
-    tq = time_kernel(lambda: mx.mxfp4_quantize(x, codes=codes, scales=scales), steps, warmup, dev, flush)
-    td = time_kernel(lambda: mx.mxfp4_dequantize(codes, scales, out=out), steps, warmup, dev, flush)
+    # copies of the 119 MB working set, cycled so that each call starts with its data
+    # out of L2 (the L2 holds 126 MB; flushing it by writes instead would leave dirty
+    # lines that the timed call then has to write back)
+    nset = -(-2 * L2_BYTES // nbytes) + 1
+    sets = [(x.clone(), torch.empty_like(codes), torch.empty_like(scales), torch.empty_like(out))
+            for _ in range(nset)]
+    tq = time_kernel(lambda i: mx.mxfp4_quantize(sets[i % nset][0], codes=sets[i % nset][1],
+                                                 scales=sets[i % nset][2]), steps, warmup, dev)
+    td = time_kernel(lambda i: mx.mxfp4_dequantize(sets[i % nset][1], sets[i % nset][2],
+                                                   out=sets[i % nset][3]), steps, warmup, dev)
     gq, gd = nbytes / tq / 1e6, nbytes / td / 1e6
     return {"workload": f"bf16 [{R}, {C}] <-> MXFP4 (1% x50 outliers, 0.5% zero blocks)",
             "bytes_per_call": nbytes,
@@ -285,8 +292,8 @@ def active_weight_bytes(cfg, logits):
     return ids, ids * per_expert
 
 
-def bench_moe_line(name, cfg, L, mode, dev, pk, flush, steps=10, warmup=3):
-    r = time_layer(L, cfg, mode, steps, warmup, dev, flush=flush)
+def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3):
+    r = time_layer(L, cfg, mode, steps, warmup, dev)
     ms = statistics.mean(r["step_ms"])
     fl = layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I)
     n_act, wbytes = active_weight_bytes(cfg, L["logits"])
@@ -311,18 +318,18 @@ def bench_moe_line(name, cfg, L, mode, dev, pk, flush, steps=10, warmup=3):
     return line
 
 
-def breakdown(dev, pk, flush):
+def breakdown(dev, pk):
     import moe_expert_gemm_mxfp4_b200 as mx
     from moe_expert_gemm_mxfp4_b200 import inputs
-    bd = {"quant": bench_quant(dev, pk, flush)}
+    bd = {"quant": bench_quant(dev, pk)}
     cfg = inputs.MOE_CONFIGS["moe_decode"]
     L = gpu_layer(cfg, dev)
-    bd["moe_decode"] = bench_moe_line("moe_decode", cfg, L, mx.W4A16, dev, pk, flush, steps=20)
+    bd["moe_decode"] = bench_moe_line("moe_decode", cfg, L, mx.W4A16, dev, pk, steps=20)
     del L
     cfg = inputs.MOE_CONFIGS["moe_120b"]
     L = gpu_layer(cfg, dev)
-    bd["moe_120b_w4a16"] = bench_moe_line("moe_120b", cfg, L, mx.W4A16, dev, pk, flush)
-    bd["moe_120b_w4a4"] = bench_moe_line("moe_120b", cfg, L, mx.W4A4, dev, pk, flush)
+    bd["moe_120b_w4a16"] = bench_moe_line("moe_120b", cfg, L, mx.W4A16, dev, pk)
+    bd["moe_120b_w4a4"] = bench_moe_line("moe_120b", cfg, L, mx.W4A4, dev, pk)
     del L
     torch.cuda.empty_cache()
     return bd
@@ -404,9 +411,19 @@ def workload_config(cfg):
                         "MXFP4 weights, W4A16",
             "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.top_k,
             "flops_per_step": layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I),
-            "l2": "256 MiB buffer written before every step (outside the per-step events); "
-                  "weights 423 MB > 126 MB L2",
+            "l2": "inputs larger than L2, no flush: every step streams all 423 MB of expert "
+                  "weights (126 MB L2); the quantize line cycles 3 copies of its 119 MB",
             "parallelism": "replicas (one layer per GPU, no collective)"}
+
+
+def kernel_source_hash():
+    """sha256[:16] over the sources of the grouped-GEMM kernels (a traffic figure
+    is only reported while these are unchanged since it was captured)."""
+    h = hashlib.sha256()
+    for name in ("common.cuh", "gemm_common.cuh", "gemm.cu", "gemm_mxf4.cu"):
+        with open(os.path.join(ROOT, "moe_expert_gemm_mxfp4_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_record(kernel, workload):
@@ -417,9 +434,7 @@ def traffic_record(kernel, workload):
         return None
     with open(path) as f:
         recs = json.load(f)
-    src = os.path.join(ROOT, "moe_expert_gemm_mxfp4_b200", "csrc", "gemm.cu")
-    with open(src, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    h = kernel_source_hash()
     r = recs.get(f"{kernel}|{workload}")
     if not r or r.get("source_sha256_16") != h:
         return None
@@ -460,11 +475,10 @@ def main():
         import dataclasses
         cfg = dataclasses.replace(cfg, T=args.tokens)
     L = gpu_layer(cfg, dev)
-    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     sampler.start()
-    r = time_layer(L, cfg, mx.W4A16, args.steps, args.warmup, dev, world=world, flush=flush)
+    r = time_layer(L, cfg, mx.W4A16, args.steps, args.warmup, dev, world=world)
     clocks = sampler.stop()
 
     fl = layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I)
@@ -504,7 +518,7 @@ def main():
     del L
     torch.cuda.empty_cache()
     if not args.no_breakdown and world == 1:
-        line["breakdown"] = breakdown(dev, pk, flush)
+        line["breakdown"] = breakdown(dev, pk)
     if not args.no_cpu and world == 1:
         line["cpu_baseline"] = cpu_baseline(cfg)
     print(json.dumps(line), flush=True)

@@ -95,7 +95,8 @@ MXFP4_API mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* sca
  * scales [N, K/32]; fp32 accumulation, one rounding to bf16 at the end.
  * Requires K % 64 == 0 and K <= 8064 (the block scales of a 128-row weight tile
  * are staged whole in shared memory); any M >= 1, N >= 1.  Workspace: W4A16 needs none
- * (ws may be NULL); W4A4 needs mxfp4_gemm_workspace_size() bytes (the quantized x). */
+ * (ws may be NULL); W4A4 needs mxfp4_gemm_workspace_size() bytes (x quantized to
+ * MXFP4: codes and block scales). */
 MXFP4_API mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K,
                         const uint8_t* w_codes, const uint8_t* w_scales, int64_t N,
                         void* y_bf16, mxfp4_mode mode, void* ws, size_t ws_bytes,
@@ -152,7 +153,8 @@ MXFP4_API size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64
  * aside on every GPU that loads the library until the process exits.
  *   - Limit: calls whose moe_mxfp4_workspace_size(...) exceeds
  *     MXFP4_NOALLOC_SCRATCH_BYTES return MXFP4_ERR_WORKSPACE (with H = I = 2880 and
- *     32 experts that is up to 724 token-expert pairs, T * top_k: decode batches).
+ *     32 experts that is up to 724 token-expert pairs, T * top_k, in W4A16 and 808
+ *     in W4A4: decode batches).
  *   - The first call on each device looks up the array's device address (a host-side
  *     query, no allocation); make that first call before any stream capture.
  *   - All calls share the one array: calls that overlap on the GPU (other streams, or

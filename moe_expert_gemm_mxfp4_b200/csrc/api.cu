@@ -122,6 +122,21 @@ mxfp4_status encode_act_map(CUtensorMap* m, const void* x, int64_t K, int64_t ro
     return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
 }
 
+// Packed E2M1 activation codes {K/2 bytes, rows}; box {128, nt} (256 K values per
+// row); 128-byte swizzle (UMMA K-major SW128 layout of a 4-bit operand).
+mxfp4_status encode_x4_map(CUtensorMap* m, const uint8_t* codes, int64_t K, int64_t rows, int nt) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(nt)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
+}
+
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace of moe_mxfp4_mlp, carved in this order (256-byte aligned pieces).
@@ -134,13 +149,22 @@ struct MoeWs {
     int32_t* inv;
     float* w_sorted;
     void* route_tmp;
-    void* x_sorted;   // bf16 [P, H]
+    void* x_sorted;   // W4A16: bf16 [P, H]
     void* h;          // bf16 [P, I]
-    void* y_sorted;   // fp32 [P, H]; W4A4 also parks the quantized x (bf16 [T, H]) here first
+    void* y_sorted;   // fp32 [P, H]
+    // W4A4 only, the MXFP4 activations: x (codes [T, H/2], scales [T, H/32]), the
+    // gathered rows (codes [P, H/2], scales [P, H/32]) and h (codes [P, I/2], scales
+    // [P, I/32]).
+    uint8_t* xq_codes;
+    uint8_t* xq_scales;
+    uint8_t* xs_codes;
+    uint8_t* xs_scales;
+    uint8_t* hq_codes;
+    uint8_t* hq_scales;
     size_t bytes;
 };
 
-MoeWs carve_moe(void* base, int64_t T, int64_t H, int64_t I, int64_t E, int top_k) {
+MoeWs carve_moe(void* base, int64_t T, int64_t H, int64_t I, int64_t E, int top_k, int mode) {
     const int64_t P = T * top_k;
     MoeWs w{};
     size_t off = 0;
@@ -157,8 +181,21 @@ MoeWs carve_moe(void* base, int64_t T, int64_t H, int64_t I, int64_t E, int top_
     w.inv = static_cast<int32_t*>(take(P * 4));
     w.w_sorted = static_cast<float*>(take(P * 4));
     w.route_tmp = take(mx::route_tmp_bytes(T, E, top_k));
-    w.x_sorted = take(static_cast<size_t>(P) * H * 2);
+    if (mode == MXFP4_W4A4) {
+        // scale arrays keep 16 readable bytes past their end (the GEMM's staging copy
+        // rounds its byte range up to 16)
+        w.xq_codes = static_cast<uint8_t*>(take(static_cast<size_t>(T) * H / 2));
+        w.xq_scales = static_cast<uint8_t*>(take(static_cast<size_t>(T) * H / 32 + 16));
+        w.xs_codes = static_cast<uint8_t*>(take(static_cast<size_t>(P) * H / 2));
+        w.xs_scales = static_cast<uint8_t*>(take(static_cast<size_t>(P) * H / 32 + 16));
+    } else {
+        w.x_sorted = take(static_cast<size_t>(P) * H * 2);
+    }
     w.h = take(static_cast<size_t>(P) * I * 2);
+    if (mode == MXFP4_W4A4) {
+        w.hq_codes = static_cast<uint8_t*>(take(static_cast<size_t>(P) * I / 2));
+        w.hq_scales = static_cast<uint8_t*>(take(static_cast<size_t>(P) * I / 32 + 16));
+    }
     w.y_sorted = take(static_cast<size_t>(P) * H * 4);
     w.bytes = off;
     return w;
@@ -224,7 +261,7 @@ mxfp4_status mxfp4_quantize(const void* x, mxfp4_in_dtype dt, int64_t rows, int6
     mxfp4_status st = device_info(&d);
     if (st != MXFP4_OK) return st;
     cudaError_t e = mx::launch_quantize(x, dt == MXFP4_IN_F32, rows, cols, codes, scales,
-                                        static_cast<int>(rule), d->sm_count,
+                                        static_cast<int>(rule), d->sm_count, d->status,
                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
@@ -240,14 +277,15 @@ mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64
     mxfp4_status st = device_info(&d);
     if (st != MXFP4_OK) return st;
     cudaError_t e = mx::launch_dequantize(codes, scales, rows, cols, out_bf16, d->sm_count,
-                                          static_cast<cudaStream_t>(stream));
+                                          d->status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
 size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp4_mode mode) {
     (void)N;
     if (mode != MXFP4_W4A4 || M <= 0 || K <= 0) return 0;
-    return align_up(static_cast<size_t>(M) * K * 2, 256);
+    return align_up(static_cast<size_t>(M) * K / 2, 256) +
+           align_up(static_cast<size_t>(M) * K / 32 + 16, 256);
 }
 
 mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t* w_codes,
@@ -257,7 +295,8 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     if (M <= 0 || K <= 0 || N <= 0) return MXFP4_ERR_INVALID_ARG;
     if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
     if (K % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
-    if (M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) || K > mx::max_gemm_k())
+    if (M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) || K > mx::max_gemm_k() ||
+        (mode == MXFP4_W4A4 && K > mx::max_gemm_k_w4a4()))
         return MXFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x_bf16) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y_bf16))
         return MXFP4_ERR_MISALIGNED;
@@ -268,16 +307,20 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     mxfp4_status st = device_info(&d);
     if (st != MXFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const void* xa = x_bf16;
-    if (mode == MXFP4_W4A4) {
-        cudaError_t e = mx::launch_qdq_bf16(x_bf16, M, K, ws, d->sm_count, s);
-        if (e != cudaSuccess) return cuda_fail(e);
-        xa = ws;
-    }
     const mx::TokenTiling tiling = mx::pick_token_tiling(M, 1);
     CUtensorMap tw, tx;
     if ((st = encode_codes_map(&tw, w_codes, K, N, 1, 128)) != MXFP4_OK) return st;
-    if ((st = encode_act_map(&tx, xa, K, M, tiling.nt)) != MXFP4_OK) return st;
+    uint8_t* xq_codes = static_cast<uint8_t*>(ws);
+    uint8_t* xq_scales = xq_codes ? xq_codes + align_up(static_cast<size_t>(M) * K / 2, 256) : nullptr;
+    if (mode == MXFP4_W4A4) {   // activations to MXFP4 (FLOOR rule, blocks along K)
+        cudaError_t e = mx::launch_quantize(x_bf16, 0, M, K, xq_codes, xq_scales, MXFP4_SCALE_FLOOR,
+                                            d->sm_count, d->status, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        st = encode_x4_map(&tx, xq_codes, K, M, tiling.nt);
+    } else {
+        st = encode_act_map(&tx, x_bf16, K, M, tiling.nt);
+    }
+    if (st != MXFP4_OK) return st;
     mx::GemmArgs a{};
     a.w_scales = w_scales;
     a.offsets = nullptr;
@@ -292,9 +335,14 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     a.n_valid_feat = static_cast<int>(N);
     a.row_w = nullptr;
     a.status = d->status;
+    a.x_scales = xq_scales;
     const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
     const int64_t tiles = ((M + tile_rows - 1) / tile_rows) * a.n_ftiles;
-    cudaError_t e = mx::launch_grouped_gemm(mx::EPI_PLAIN, tiling, tw, tx, a, gemm_grid(d, tiles), s);
+    cudaError_t e = mode == MXFP4_W4A4
+                        ? mx::launch_grouped_gemm_w4a4(mx::EPI_PLAIN, tiling.nt, tw, tx, a,
+                                                       gemm_grid(d, tiles), s)
+                        : mx::launch_grouped_gemm(mx::EPI_PLAIN, tiling, tw, tx, a,
+                                                  gemm_grid(d, tiles), s);
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
@@ -326,16 +374,15 @@ mxfp4_status moe_mxfp4_route(const float* router_logits, int64_t T, int64_t E, i
     DeviceInfo* d = nullptr;
     if ((st = device_info(&d)) != MXFP4_OK) return st;
     cudaError_t e = mx::launch_route(router_logits, T, E, top_k, ids, weights, counts, offsets, perm,
-                                     inv, nullptr, ws, nullptr, 0, nullptr, d->sm_count,
-                                     static_cast<cudaStream_t>(stream));
+                                     inv, nullptr, ws, nullptr, 0, nullptr, nullptr, 0, nullptr,
+                                     d->sm_count, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
 size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k,
                                 mxfp4_mode mode) {
-    (void)mode;
     if (T <= 0 || H <= 0 || I <= 0 || E <= 0 || top_k <= 0) return 0;
-    return carve_moe(nullptr, T, H, I, E, top_k).bytes;
+    return carve_moe(nullptr, T, H, I, E, top_k, mode).bytes;
 }
 
 mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float* router_logits,
@@ -351,6 +398,8 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
     if (H % 64 != 0 || I % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
     if (H > mx::max_gemm_k() || I > mx::max_gemm_k()) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (mode == MXFP4_W4A4 && (H > mx::max_gemm_k_w4a4() || I > mx::max_gemm_k_w4a4()))
+        return MXFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x_bf16) || !aligned16(router_logits) || !aligned16(w13_codes) ||
         !aligned16(w13_scales) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
         !aligned16(out_bf16))
@@ -361,21 +410,27 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     DeviceInfo* d = nullptr;
     if ((st = device_info(&d)) != MXFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const MoeWs w = carve_moe(ws, T, H, I, E, top_k);
+    const MoeWs w = carve_moe(ws, T, H, I, E, top_k, mode);
     const int64_t P = T * top_k;
     cudaError_t e;
 
     trace_mark(0, s);
-    const void* x_src = x_bf16;
-    if (mode == MXFP4_W4A4) {   // activations on the MXFP4 grid, rows along H
-        if ((e = mx::launch_qdq_bf16(x_bf16, T, H, w.y_sorted, d->sm_count, s)) != cudaSuccess)
+    const bool a4 = mode == MXFP4_W4A4;
+    if (a4) {
+        // W4A4: x to MXFP4 per token (FLOOR rule, blocks along H); the gather then
+        // moves packed rows (H/2 code bytes + H/32 scale bytes) instead of bf16 rows
+        if ((e = mx::launch_quantize(x_bf16, 0, T, H, w.xq_codes, w.xq_scales, MXFP4_SCALE_FLOOR,
+                                     d->sm_count, d->status, s)) != cudaSuccess)
             return cuda_fail(e);
-        x_src = w.y_sorted;
+        e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets,
+                             w.perm, w.inv, w.w_sorted, w.route_tmp, w.xq_codes, H / 2, w.xs_codes,
+                             w.xq_scales, H / 32, w.xs_scales, d->sm_count, s);
+    } else {
+        e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets,
+                             w.perm, w.inv, w.w_sorted, w.route_tmp, x_bf16, H * 2, w.x_sorted,
+                             nullptr, 0, nullptr, d->sm_count, s);
     }
-    if ((e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets,
-                              w.perm, w.inv, w.w_sorted, w.route_tmp, x_src, H, w.x_sorted,
-                              d->sm_count, s)) != cudaSuccess)
-        return cuda_fail(e);
+    if (e != cudaSuccess) return cuda_fail(e);
 
     trace_mark(1, s);
     const mx::TokenTiling tiling = mx::pick_token_tiling(P, E);
@@ -384,10 +439,13 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
 
     // gate/up projection with the SwiGLU epilogue -> h [P, I]
     CUtensorMap tw, tx;
-    if ((st = encode_codes_map(&tw, w13_codes, H, 2 * I, E, 64)) != MXFP4_OK) return st;
-    if ((st = encode_act_map(&tx, w.x_sorted, H, P, tiling.nt)) != MXFP4_OK) return st;
+    if ((st = encode_codes_map(&tw, w13_codes, H, 2 * I, E, a4 ? 16 : 64)) != MXFP4_OK) return st;
+    st = a4 ? encode_x4_map(&tx, w.xs_codes, H, P, tiling.nt)
+            : encode_act_map(&tx, w.x_sorted, H, P, tiling.nt);
+    if (st != MXFP4_OK) return st;
     mx::GemmArgs a{};
     a.w_scales = w13_scales;
+    a.x_scales = w.xs_scales;
     a.offsets = w.offsets;
     a.m_single = 0;
     a.G = static_cast<int>(E);
@@ -400,20 +458,25 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     a.n_valid_feat = static_cast<int>(I);
     a.row_w = nullptr;
     a.status = d->status;
-    if ((e = mx::launch_grouped_gemm(mx::EPI_SWIGLU, tiling, tw, tx, a,
-                                     gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
-        return cuda_fail(e);
+    const int grid1 = gemm_grid(d, tok_tiles * a.n_ftiles);
+    e = a4 ? mx::launch_grouped_gemm_w4a4(mx::EPI_SWIGLU, tiling.nt, tw, tx, a, grid1, s)
+           : mx::launch_grouped_gemm(mx::EPI_SWIGLU, tiling, tw, tx, a, grid1, s);
+    if (e != cudaSuccess) return cuda_fail(e);
 
     trace_mark(2, s);
-    if (mode == MXFP4_W4A4) {   // h on the MXFP4 grid, rows along I (in place)
-        if ((e = mx::launch_qdq_bf16(w.h, P, I, w.h, d->sm_count, s)) != cudaSuccess)
+    if (a4) {   // h to MXFP4 (FLOOR rule, blocks along I)
+        if ((e = mx::launch_quantize(w.h, 0, P, I, w.hq_codes, w.hq_scales, MXFP4_SCALE_FLOOR,
+                                     d->sm_count, d->status, s)) != cudaSuccess)
             return cuda_fail(e);
     }
 
     // down projection, routing weight applied in fp32 -> y_sorted fp32 [P, H]
     if ((st = encode_codes_map(&tw, w2_codes, I, H, E, 128)) != MXFP4_OK) return st;
-    if ((st = encode_act_map(&tx, w.h, I, P, tiling.nt)) != MXFP4_OK) return st;
+    st = a4 ? encode_x4_map(&tx, w.hq_codes, I, P, tiling.nt)
+            : encode_act_map(&tx, w.h, I, P, tiling.nt);
+    if (st != MXFP4_OK) return st;
     a.w_scales = w2_scales;
+    a.x_scales = w.hq_scales;
     a.K = static_cast<int>(I);
     a.rows_w = static_cast<int>(H);
     a.I = 0;
@@ -422,9 +485,10 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     a.out_ld = H;
     a.n_valid_feat = static_cast<int>(H);
     a.row_w = w.w_sorted;
-    if ((e = mx::launch_grouped_gemm(mx::EPI_WEIGHTED, tiling, tw, tx, a,
-                                     gemm_grid(d, tok_tiles * a.n_ftiles), s)) != cudaSuccess)
-        return cuda_fail(e);
+    const int grid2 = gemm_grid(d, tok_tiles * a.n_ftiles);
+    e = a4 ? mx::launch_grouped_gemm_w4a4(mx::EPI_WEIGHTED, tiling.nt, tw, tx, a, grid2, s)
+           : mx::launch_grouped_gemm(mx::EPI_WEIGHTED, tiling, tw, tx, a, grid2, s);
+    if (e != cudaSuccess) return cuda_fail(e);
 
     trace_mark(3, s);
     // deterministic combine in slot order

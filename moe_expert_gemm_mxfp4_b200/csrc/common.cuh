@@ -147,6 +147,32 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= (A . 2^SFA) * (B . 2^SFB)^T, kind::mxf4 with one E8M0 scale per 32
+// K-elements of each operand (scale_vec::2X): A and B are packed E2M1 tiles in
+// shared memory (K-major, 128B swizzle), K = 64 per instruction, fp32 D in TMEM.
+// sfa / sfb are the TMEM addresses of the scale bytes; bits 30-31 carry the byte
+// within the 32-bit column (the scale id), which the instruction descriptor repeats.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Shared memory -> TMEM: a 32-row x 128-bit matrix (rows 16 B apart) into four
+// consecutive 32-bit columns of lanes 0-31, repeated in each of the four lane
+// quarters (lanes 32q + r get row r).  Ordered with the issuing thread's later
+// tcgen05.mma like any tcgen05 operation of that thread.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -218,6 +244,29 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory descriptor of an unswizzled K-major matrix made of 8-row core
+// matrices (8 rows x 16 B, 128 B each) that follow each other: start address >> 4
+// (bits 0-13), leading byte offset 16 >> 4 (bits 16-29; one core matrix along K,
+// not used), stride byte offset 128 >> 4 (bits 32-45), version 1 (bits 46-47),
+// layout type 0 = no swizzle (bits 61-63).
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(16 >> 4) << 16;
+    d |= static_cast<uint64_t>(128 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    return d;
+}
+
+// Instruction descriptor of kind::mxf4.block_scale: B scale id (bits 4-5), A and B
+// formats E2M1 (bits 7-9, 10-12: 1), both K-major (bits 15, 16: 0), N >> 3 (bits
+// 17-22), scale format E8M0 (bit 23: 1), M >> 4 (bits 24-28), A scale id (bits
+// 29-30), K = 64 (bit 31: 0).  D is fp32.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sf_id) {
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(M >> 4) << 24) | (sf_id << 29);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -35,27 +35,30 @@
 // TMEM: columns [0, 256) accumulators (TT*NT columns per buffer, double-buffered
 // when they fit), [256, 512) eight 32-column A slots.
 // Every mbarrier wait is time-bounded (MXFP4_ERR_TIMEOUT in the status word).
-#include "common.cuh"
-#include "internal.h"
+#include "gemm_common.cuh"
 
 namespace mx {
 
 namespace {
 
+using namespace gemm;
+
 constexpr int kThreads = 512;
-constexpr int kBM = 128;            // weight rows per tile (MMA M)
 constexpr int kBK = 64;             // K per pipeline stage
 constexpr int kASlots = 8;          // TMEM A-operand slots (32 columns each)
 constexpr int kACol0 = 256;         // first TMEM column of the A slots
 constexpr int kSub = 4;             // 64-wide K sub-stages per codes super-stage
 constexpr int kCodeRowBytes = kSub * kBK / 2;          // 128 B of codes per weight row
 constexpr int kCodeBytes = kBM * kCodeRowBytes;        // one codes super-stage (16 KB)
-constexpr int kLutBytes = 256 * 256;
-constexpr int kMaxGroups = 256;
+constexpr int kLutBytes = 256 * 256;   // 256 byte values x 256-B rows (32 lanes x bf16x2 used)
 constexpr int kXbufBytes = 0;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxRing = 16;
 constexpr int kMaxCodeStages = 4;
+// Small token tiles (decode) stream weights at a far higher rate per MMA: their codes
+// ring takes the shared memory the activation ring leaves free (up to 8 x 16 KB in
+// flight per SM keeps HBM busy at ~1.5 us of latency).
+constexpr int kMaxCodeStagesLock = 8;
 
 template <int NT, int TT>
 struct Cfg {
@@ -67,7 +70,7 @@ struct Cfg {
     // NT <= 64: the activation ring has one stage per A slot and both are released by
     // the same MMA commit (one commit per K stage instead of two).
     static constexpr bool kLock = NT <= 64;
-    static constexpr int kMaxActStages = kLock ? kASlots : (TT == 1 ? 5 : 3);
+    static constexpr int kMaxActStages = kLock ? kASlots : (TT == 1 ? 5 : kSub);
     static constexpr int kChunk = kAccCols < 32 ? kAccCols : 32;   // epilogue columns per TMEM load
     static_assert(kActTile % 1024 == 0, "activation tiles must keep 1024-B alignment");
     static_assert(kAccCols <= kACol0, "accumulators overlap the A slots");
@@ -96,18 +99,6 @@ __host__ __device__ inline Layout make_layout(int act_stage_bytes, int code_stag
     return L;
 }
 
-// Position in a ring of n slots with the parity of the slot's current use.
-struct Ring {
-    int idx = 0;
-    uint32_t ph = 0;
-    __device__ __forceinline__ void next(int n) {
-        if (++idx == n) {
-            idx = 0;
-            ph ^= 1u;
-        }
-    }
-};
-
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -120,27 +111,15 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-    uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr));
-    return v;
-}
-
 // 16 code bytes (32 weights of one K block) -> 16 bf16x2 words.
 // Fast path (S in [2, 254]): LUT value times 2^(S-127) as one bf16x2 multiply,
 // exact because both factors and the product are normal bf16 numbers (or the
 // product overflows to Inf, as round-to-nearest-even does).  Otherwise the
 // exact fp32 route (subnormal results for S <= 1, NaN for S = 255).
-// LUT entry (b, lane) sits at lut_base + b * 256 + lane * 4; lut_lane is
-// lut_base + lane * 4 and prmt places code byte j of a word at bits 8..15.
+// LUT entry (b, lane) sits at lut_base + b * 256 + lane * 4 (lane-replicated, so
+// the 32 lanes of a warp hit 32 different banks whatever their bytes); lut_lane
+// is lut_base + lane * 4 and one prmt places code byte j of a word at bits 8..15,
+// which makes the row address b * 256 without a multiply.
 __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lut_lane,
                                                 uint32_t* out) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
@@ -161,62 +140,6 @@ __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lu
 #pragma unroll
             for (int j = 0; j < 4; ++j) out[4 * i + j] = dequant_byte_exact((w[i] >> (8 * j)) & 0xFFu, sc);
     }
-}
-
-__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
-
-__device__ __forceinline__ void store_bf16(void* out, int64_t idx, float v) {
-    reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-}
-
-// Copy `rows` consecutive rows of block scales (kb bytes each) from global to
-// shared: the 16-byte multiple with one bulk copy (counted on `bar`), the tail
-// with plain loads.  Returns the bulk byte count.
-__device__ __forceinline__ uint32_t stage_scales(uint8_t* dst, const uint8_t* src, int rows, int kb,
-                                                 uint64_t* bar) {
-    const uint32_t bytes = static_cast<uint32_t>(rows * kb);
-    const uint32_t bulk = bytes & ~15u;
-    if (bulk) bulk_load(dst, src, bulk, bar);
-    if (bulk < bytes) {
-        for (uint32_t i = bulk; i < bytes; ++i) dst[i] = src[i];
-        // order these generic-proxy writes before later bulk copies into the buffer
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    return bulk;
-}
-
-struct TileInfo {
-    int g, f, row0, mrows;
-};
-
-// The ki-th 64-wide K stage of a tile when its super-stages are visited starting at
-// super-stage `rot` (the last super-stage may hold fewer than kSub stages).
-__device__ __forceinline__ int stage_at(int ki, int rot, int nss, int nk) {
-    const int rot_stage = rot * kSub;              // stages visited before wrapping
-    const int first = nk - rot_stage;              // stages from super-stage rot to the end
-    return ki < first ? rot_stage + ki : ki - first;
-}
-
-// Work tile t -> (group, feature tile, first row, valid rows).  Tiles of a group
-// are numbered feature-tile-major with the token tile fastest, so CTAs working at
-// the same time share the weight tile (L2 reuse).
-__device__ __forceinline__ TileInfo decode_tile(int t, const int* s_tstart, const int* s_off, int G,
-                                                int tile_rows) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {                 // largest g with s_tstart[g] <= t
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_tstart[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    TileInfo ti;
-    ti.g = lo;
-    const int m = s_off[lo + 1] - s_off[lo];
-    const int mt = (m + tile_rows - 1) / tile_rows;
-    const int local = t - s_tstart[lo];
-    ti.f = local / mt;
-    const int tt = local - ti.f * mt;
-    ti.row0 = s_off[lo] + tt * tile_rows;
-    ti.mrows = min(tile_rows, m - tt * tile_rows);
-    return ti;
 }
 
 template <int NT, int TT, int MODE>
@@ -318,7 +241,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     if (warp == 0) {
         // ---------------- codes (+ scales) producer
         if (lane == 0) {
-            Ring c;
+            RingPos c;
             int lt = 0, issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
@@ -360,7 +283,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 *s_abort = 1;
                 record_status(args.status, MXFP4_ERR_TIMEOUT);
                 // let the copies already issued land before the CTA exits
-                Ring r;
+                RingPos r;
                 const int first = issued > SC ? issued - SC : 0;
                 for (int i = 0; i < issued; ++i) {
                     if (i >= first) mbar_wait(&cfull[r.idx], r.ph, s_never);
@@ -373,7 +296,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     } else if (warp == 2) {
         // ---------------- activation producer
         if (lane == 0) {
-            Ring x;             // kLock: ring of A-slot sets (2); else: ring of stages (SA)
+            RingPos x;             // kLock: ring of A-slot sets (2); else: ring of stages (SA)
             int issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
@@ -417,7 +340,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 record_status(args.status, MXFP4_ERR_TIMEOUT);
                 // let the copies already issued land before the CTA exits
                 if (C::kLock) {
-                    Ring r;
+                    RingPos r;
                     const int first = issued > 2 ? issued - 2 : 0;
                     for (int i = 0; i < issued; ++i) {
                         if (i >= first)
@@ -425,7 +348,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         r.next(2);
                     }
                 } else {
-                    Ring r;
+                    RingPos r;
                     const int first = issued > SA ? issued - SA : 0;
                     for (int i = 0; i < issued; ++i) {
                         if (i >= first) mbar_wait(&xfull[r.idx], r.ph, s_never);
@@ -441,7 +364,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         // of the MMAs in flight, so it is paid once per group, not once per stage.
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kBM, NT);
-            Ring x, a;          // x: activation stages (only when !kLock); a: A-slot sets
+            RingPos x, a;          // x: activation stages (only when !kLock); a: A-slot sets
             int lt = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
@@ -502,7 +425,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         }
         const uint32_t sw = static_cast<uint32_t>(srow) & 7u;   // 128B swizzle: chunk ^= row % 8
         const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
-        Ring c, a, xr;        // codes super-stages, A-slot sets, activation stages (!kLock)
+        RingPos c, a, xr;        // codes super-stages, A-slot sets, activation stages (!kLock)
         int kit = 0, lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
@@ -558,9 +481,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     } else if (warp >= 12) {
         // ---------------- epilogue warpgroup
         constexpr int CW = C::kChunk;
-        constexpr int NCH = C::kAccCols / CW;
         const int q = warp & 3;
-        const bool lo = lane < 16;
         int lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
@@ -570,58 +491,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&accfull[b], bph, s_abort))) { ok = false; break; }
             tc_fence_after();
             const uint32_t t_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::kAccCols;
-            // column j of the accumulator set is token row ti.row0 + j
-            auto process = [&](const uint32_t* cur, int c) {
-                if (MODE == EPI_SWIGLU) {
-                    // lanes < 16 finish columns [0, CW/2) of the chunk, lanes >= 16 columns
-                    // [CW/2, CW); each needs its partner's (lane ^ 16) gate or up value
-                    const int feat = ti.f * 64 + 16 * q + (lane & 15);
-#pragma unroll
-                    for (int i = 0; i < CW / 2; ++i) {
-                        const uint32_t send = lo ? cur[CW / 2 + i] : cur[i];
-                        const float other = __uint_as_float(__shfl_xor_sync(0xFFFFFFFFu, send, 16));
-                        const float g = lo ? __uint_as_float(cur[i]) : other;
-                        const float u = lo ? other : __uint_as_float(cur[CW / 2 + i]);
-                        const int tok = c * CW + (lo ? i : CW / 2 + i);
-                        if (tok < ti.mrows)
-                            store_bf16(args.out, static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat,
-                                       silu_f32(g) * u);
-                    }
-                } else {
-                    const int feat = ti.f * kBM + q * 32 + lane;
-                    if (feat < args.n_valid_feat) {
-#pragma unroll
-                        for (int n = 0; n < CW; ++n) {
-                            const int tok = c * CW + n;
-                            if (tok < ti.mrows) {
-                                const int64_t idx = static_cast<int64_t>(ti.row0 + tok) * args.out_ld + feat;
-                                const float val = __uint_as_float(cur[n]);
-                                if (MODE == EPI_WEIGHTED)   // fp32 out: one rounding, in the combine
-                                    reinterpret_cast<float*>(args.out)[idx] = val * args.row_w[ti.row0 + tok];
-                                else
-                                    store_bf16(args.out, idx, val);
-                            }
-                        }
-                    }
-                }
-            };
-            auto load = [&](uint32_t* dst, int c) {
-                if (CW == 32) tmem_ld_x32(t_base + c * CW, dst); else tmem_ld_x16(t_base + c * CW, dst);
-            };
-            // two register buffers: the next chunk's TMEM load overlaps this chunk's work
-            uint32_t v0[CW], v1[CW];
-            load(v0, 0);
-#pragma unroll 1
-            for (int c = 0; c < NCH; c += 2) {
-                tmem_wait_ld();
-                if (c + 1 < NCH) load(v1, c + 1);
-                process(v0, c);
-                if (c + 1 < NCH) {
-                    tmem_wait_ld();
-                    if (c + 2 < NCH) load(v0, c + 2);
-                    process(v1, c + 1);
-                }
-            }
+            epilogue_tile<MODE, CW, C::kAccCols>(args, ti, t_base, q, lane);
             tc_fence_before();
             mbar_arrive(&accempty[b]);
         }
@@ -646,7 +516,7 @@ bool ring_depths(int K, int* sc, int* sa, int* smem) {
     using C = Cfg<NT, TT>;
     // The activation ring must hold at least one whole group of kSub stages: the MMA
     // issuer consumes a group only once all its stages are ready.
-    int c = kMaxCodeStages, a = C::kMaxActStages;
+    int c = C::kLock ? kMaxCodeStagesLock : kMaxCodeStages, a = C::kMaxActStages;
     while (make_layout(C::kActStage, c, a, K).total > kSmemLimit) {
         if (c > 2) --c;
         else if (!C::kLock && a > kSub) --a;
@@ -678,7 +548,10 @@ cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap
     if (nt == 16) return launch_cfg<16, 1, MODE>(tw, tx, a, grid, stream);
     if (nt == 32) return launch_cfg<32, 1, MODE>(tw, tx, a, grid, stream);
     if (nt == 64) return launch_cfg<64, 1, MODE>(tw, tx, a, grid, stream);
-    (void)tt;
+    if (tt == 2) {   // two token tiles per weight tile when their rings fit this K
+        int sc, sa, smem;
+        if (ring_depths<128, 2>(a.K, &sc, &sa, &smem)) return launch_cfg<128, 2, MODE>(tw, tx, a, grid, stream);
+    }
     return launch_cfg<128, 1, MODE>(tw, tx, a, grid, stream);
 }
 

@@ -24,6 +24,7 @@ struct GemmArgs {
     int64_t out_ld;            // elements per output row
     int n_valid_feat;          // valid output columns
     const float* row_w;        // WEIGHTED: per-row scalar
+    const uint8_t* x_scales;   // W4A4: activation block scales [rows, K/32] (+16 readable bytes)
     unsigned* status;          // device status word
     int code_stages;           // ring depths (set by launch_grouped_gemm)
     int act_stages;
@@ -38,16 +39,16 @@ struct TokenTiling {
 
 cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t cols,
                             uint8_t* codes, uint8_t* scales, int rule, int sm_count,
-                            cudaStream_t stream);
-cudaError_t launch_qdq_bf16(const void* x, int64_t rows, int64_t cols, void* out, int sm_count,
-                            cudaStream_t stream);
+                            unsigned* status, cudaStream_t stream);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
-                              int64_t cols, void* out, int sm_count, cudaStream_t stream);
+                              int64_t cols, void* out, int sm_count, unsigned* status,
+                              cudaStream_t stream);
 size_t route_tmp_bytes(int64_t T, int64_t E, int top_k);
 cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, int32_t* ids,
                          float* weights, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv, float* w_sorted, void* tmp, const void* x, int64_t H,
-                         void* x_sorted, int sm_count, cudaStream_t stream);
+                         int32_t* inv, float* w_sorted, void* tmp, const void* x,
+                         int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
+                         void* xs_sorted, int sm_count, cudaStream_t stream);
 cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, int top_k,
                            int64_t H, void* out, int sm_count, cudaStream_t stream);
 TokenTiling pick_token_tiling(int64_t rows, int64_t groups);
@@ -55,5 +56,9 @@ int64_t max_gemm_k();   // largest contraction length the grouped GEMM accepts
 cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream);
+int64_t max_gemm_k_w4a4();   // largest contraction length the W4A4 engine accepts
+cudaError_t launch_grouped_gemm_w4a4(int mode, int nt, const CUtensorMap& tmap_w,
+                                     const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
+                                     cudaStream_t stream);
 
 }  // namespace mx

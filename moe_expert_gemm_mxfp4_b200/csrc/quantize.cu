@@ -7,14 +7,18 @@
 // element, Inf/NaN blocks -> scale 0xFF) are documented in include/mxfp4.h.
 //
 // Layout of the work: the input is treated as a flat array of 32-element blocks
-// (cols % 32 == 0, so blocks never straddle rows).  One warp handles 32 blocks
-// per step: 128-bit coalesced loads spread each block over 4 lanes (bf16) or 8
-// lanes (fp32); the block amax is a shuffle reduction over those lanes; the
-// scale is pure integer work on the amax bit pattern; |v| / 2^s is an exact
-// power-of-two product in fp32 and the E2M1 rounding is the hardware
-// cvt.rn.satfinite.e2m1x2.f32 (round-to-nearest-even, saturating at 6).  Codes
-// are staged through shared memory so that each lane stores one whole block
-// (16 bytes) with a 128-bit store.
+// (cols % 32 == 0, so blocks never straddle rows), cut into chunks of
+// consecutive blocks.  Each CTA is persistent over chunks c = blockIdx.x,
+// blockIdx.x + gridDim.x, ...: one producer thread streams its chunks into a
+// ring of shared-memory stages with cp.async.bulk (completion counted on an
+// mbarrier per stage), so that a whole ring of bytes per CTA is in flight from
+// HBM; eight consumer warps convert a stage and release it.  Quantize: 128-bit
+// shared-memory reads spread each block over 4 lanes (bf16) or 8 lanes (fp32);
+// the block amax is a shuffle reduction over those lanes; the scale is pure
+// integer work on the amax bit pattern; |v| / 2^s is an exact power-of-two
+// product in fp32 and the E2M1 rounding is the hardware
+// cvt.rn.satfinite.e2m1x2.f32 (round-to-nearest-even, saturating at 6).
+// Dequantize: each lane expands 4 code bytes to 8 bf16 values exactly.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,8 +26,6 @@ namespace mx {
 
 namespace {
 
-constexpr int kQThreads = 256;
-constexpr int kWarpsPerCta = kQThreads / 32;
 
 // Block exponent s from the amax magnitude bits of a bf16 block.
 __device__ __forceinline__ int block_exp_bf16(uint32_t amax, int rule) {
@@ -122,29 +124,118 @@ __device__ __forceinline__ uint4 dequant8(uint32_t cw, uint32_t S) {
     return o;
 }
 
+// ---------------------------------------------------------------- bulk-copy ring
+// Stage ring shared by the streaming kernels: full[i] completes when stage i's
+// bulk copies have landed, empty[i] when all consumer warps have read it.
+constexpr int kRingConsumerWarps = 8;
+constexpr int kRingThreads = (kRingConsumerWarps + 1) * 32;   // + one producer warp
+constexpr int kRingCtasPerSm = 2;
+constexpr int kRingMaxStages = 8;
+constexpr int kRingSmemBytes = 96 * 1024;                      // per CTA
+
+struct Ring {
+    uint64_t full[kRingMaxStages];
+    uint64_t empty[kRingMaxStages];
+    int abort;
+};
+
+__device__ __forceinline__ void ring_init(Ring& r, int n_stages) {
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < n_stages; ++i) {
+            mbar_init(&r.full[i], 1);
+            mbar_init(&r.empty[i], kRingConsumerWarps);
+        }
+        r.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+}
+
+// Producer (one thread): for each chunk of this CTA wait for a free stage, then
+// `issue(stage, chunk, bar)` posts the bulk copies (arrive.expect_tx + copies).
+// On abort or timeout it stops issuing; before returning it waits (bounded) for
+// every copy it posted, so that no copy lands in shared memory after exit.
+template <class Issue>
+__device__ __forceinline__ void ring_produce(Ring& r, int n_stages, int64_t n_chunks, Issue issue,
+                                             unsigned* status) {
+    int st = 0;
+    uint32_t ph = 0;
+    uint32_t posted = 0, last_ph = 0;   // bit i: stage i holds a copy posted in phase bit i of last_ph
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        if (!mbar_wait(&r.empty[st], ph ^ 1u, &r.abort)) {
+            if (!r.abort) record_status(status, MXFP4_ERR_TIMEOUT);
+            r.abort = 1;
+            break;
+        }
+        issue(st, c, &r.full[st]);
+        posted |= 1u << st;
+        last_ph = (last_ph & ~(1u << st)) | (ph << st);
+        if (++st == n_stages) {
+            st = 0;
+            ph ^= 1u;
+        }
+    }
+    if (r.abort) {
+        int never = 0;
+        for (int i = 0; i < n_stages; ++i)
+            if ((posted >> i) & 1u) (void)mbar_wait(&r.full[i], (last_ph >> i) & 1u, &never);
+    }
+}
+
+// Consumer side of one stage: wait until it is full (bounded).
+__device__ __forceinline__ bool ring_wait_full(Ring& r, int st, uint32_t ph, unsigned* status) {
+    if (mbar_wait(&r.full[st], ph, &r.abort)) return true;
+    if (!r.abort) record_status(status, MXFP4_ERR_TIMEOUT);
+    r.abort = 1;
+    return false;
+}
+
+// Consumer warp done reading stage st.
+__device__ __forceinline__ void ring_release(Ring& r, int st) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&r.empty[st]);
+}
+
 // ---------------------------------------------------------------- bf16 -> MXFP4
-// One warp step = 128 uint4 vectors = 32 blocks.  Lane l loads vectors
-// 32j + l (j = 0..3); block 8j + l/4 therefore lives on lanes 4(l/4) .. +3.
-// If `qdq_out` is set, the kernel writes the dequantized bf16 values instead of
-// codes/scales (fake quantization for the W4A4 path).
-__global__ void __launch_bounds__(kQThreads)
-quantize_bf16_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint4* __restrict__ codes,
-                     uint8_t* __restrict__ scales, int rule, uint4* __restrict__ qdq_out) {
-    __shared__ __align__(16) uint32_t s_codes[kWarpsPerCta][128];
-    __shared__ uint8_t s_scales[kWarpsPerCta][32];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int64_t n_vec = n_blocks * 4;
-    const int64_t n_steps = (n_blocks + 31) >> 5;
-    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t step = warp0; step < n_steps; step += nwarps) {
-        const int64_t vbase = step * 128;
+// Chunk = 256 blocks (16 KB of bf16).  Consumer warp w converts blocks
+// 32w .. 32w+31 of the chunk: lane l reads vectors 32j + l (j = 0..3) of the
+// warp's 2 KB, so block 8j + l/4 lives on lanes 4(l/4) .. +3, and each lane
+// writes the 4 code bytes of its vector (a warp store covers 128 contiguous
+// bytes).  The 32 scale bytes are gathered by shuffles so that lane l stores
+// block l's.
+constexpr int kChunkBlocks = 256;
+
+__global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
+quantize_bf16_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint32_t* __restrict__ codes,
+                     uint8_t* __restrict__ scales, int rule, unsigned* status) {
+    constexpr int kStageBytes = kChunkBlocks * 64;
+    constexpr int kStages = kRingSmemBytes / kStageBytes;   // 6
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ Ring ring;
+    ring_init(ring, kStages);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t n_chunks = (n_blocks + kChunkBlocks - 1) / kChunkBlocks;
+    if (warp == kRingConsumerWarps) {
+        if (lane == 0)
+            ring_produce(ring, kStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
+                const int64_t nb = min(static_cast<int64_t>(kChunkBlocks), n_blocks - c * kChunkBlocks);
+                const uint32_t bytes = static_cast<uint32_t>(nb * 64);
+                mbar_arrive_expect_tx(bar, bytes);
+                bulk_load(smem + st * kStageBytes, x + c * kStageBytes, bytes, bar);
+            }, status);
+        return;
+    }
+    int st = 0;
+    uint32_t ph = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        if (!ring_wait_full(ring, st, ph, status)) break;
+        const uint4* src = reinterpret_cast<const uint4*>(smem + st * kStageBytes) + warp * 128;
         uint4 v[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t idx = vbase + 32 * j + lane;
-            v[j] = idx < n_vec ? __ldcs(x + idx) : make_uint4(0, 0, 0, 0);
-        }
+        for (int j = 0; j < 4; ++j) v[j] = src[32 * j + lane];
+        ring_release(ring, st);
+        const int64_t blk0 = c * kChunkBlocks + warp * 32;   // first block of this warp
+        uint32_t mine = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             uint32_t nf = 0;
@@ -156,45 +247,58 @@ quantize_bf16_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint4* __res
             const int s = block_exp_bf16(am, rule);
             const uint32_t cw = nf ? 0u : quant8_bf16(v[j], inv_pow2(s));
             const uint32_t S = nf ? 0xFFu : static_cast<uint32_t>(s + 127);
-            if (qdq_out) {
-                const int64_t idx = vbase + 32 * j + lane;
-                if (idx < n_vec) qdq_out[idx] = dequant8(cw, S);
-            } else {
-                s_codes[wid][32 * j + lane] = cw;
-                if ((lane & 3) == 0) s_scales[wid][8 * j + (lane >> 2)] = static_cast<uint8_t>(S);
-            }
+            const int64_t blk = blk0 + 8 * j + (lane >> 2);
+            if (blk < n_blocks) __stcs(codes + blk0 * 4 + 32 * j + lane, cw);
+            // block 8j + q (q = 0..7) lives on lanes 4q .. 4q+3; lane 8j + q takes its scale
+            const uint32_t got = __shfl_sync(0xFFFFFFFFu, S, (lane & 7) * 4);
+            if ((lane >> 3) == j) mine = got;
         }
-        if (!qdq_out) {
-            __syncwarp();
-            const int64_t blk = step * 32 + lane;
-            if (blk < n_blocks) {
-                codes[blk] = reinterpret_cast<const uint4*>(s_codes[wid])[lane];
-                scales[blk] = s_scales[wid][lane];
-            }
-            __syncwarp();
+        if (blk0 + lane < n_blocks) scales[blk0 + lane] = static_cast<uint8_t>(mine);
+        if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
         }
     }
 }
 
 // ---------------------------------------------------------------- fp32 -> MXFP4
-// One warp step = 256 uint4 vectors (4 fp32 each) = 32 blocks; a block spans 8 lanes.
-__global__ void __launch_bounds__(kQThreads)
-quantize_f32_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint4* __restrict__ codes,
-                    uint8_t* __restrict__ scales, int rule) {
-    __shared__ __align__(16) uint16_t s_codes[kWarpsPerCta][256];
-    __shared__ uint8_t s_scales[kWarpsPerCta][32];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int64_t n_vec = n_blocks * 8;
-    const int64_t n_steps = (n_blocks + 31) >> 5;
-    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t step = warp0; step < n_steps; step += nwarps) {
-        const int64_t vbase = step * 256;
-#pragma unroll 2
+// Chunk = 256 blocks (32 KB of fp32).  Consumer warp w converts blocks
+// 32w .. 32w+31: step j (0..7) reads vectors 32j + l, i.e. block 4j + l/8, a
+// block spanning 8 lanes; each lane produces 2 code bytes.
+__global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
+quantize_f32_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint16_t* __restrict__ codes,
+                    uint8_t* __restrict__ scales, int rule, unsigned* status) {
+    constexpr int kStageBytes = kChunkBlocks * 128;
+    constexpr int kStages = kRingSmemBytes / kStageBytes;   // 3
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ Ring ring;
+    ring_init(ring, kStages);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t n_chunks = (n_blocks + kChunkBlocks - 1) / kChunkBlocks;
+    if (warp == kRingConsumerWarps) {
+        if (lane == 0)
+            ring_produce(ring, kStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
+                const int64_t nb = min(static_cast<int64_t>(kChunkBlocks), n_blocks - c * kChunkBlocks);
+                const uint32_t bytes = static_cast<uint32_t>(nb * 128);
+                mbar_arrive_expect_tx(bar, bytes);
+                bulk_load(smem + st * kStageBytes, x + c * kStageBytes, bytes, bar);
+            }, status);
+        return;
+    }
+    int st = 0;
+    uint32_t ph = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        if (!ring_wait_full(ring, st, ph, status)) break;
+        const uint4* src = reinterpret_cast<const uint4*>(smem + st * kStageBytes) + warp * 256;
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = src[32 * j + lane];
+        ring_release(ring, st);
+        const int64_t blk0 = c * kChunkBlocks + warp * 32;
+        uint32_t mine = 0;
+#pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int64_t idx = vbase + 32 * j + lane;
-            const uint4 v = idx < n_vec ? __ldcs(x + idx) : make_uint4(0, 0, 0, 0);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
             uint32_t am = 0, nf = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -209,103 +313,137 @@ quantize_f32_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint4* __rest
             }
             const int s = block_exp_f32(am, rule);
             const float mult = inv_pow2(s);
-            uint32_t c;
-            {
-                uint32_t b;
-                asm("{\n\t.reg .b8 b0, b1;\n\t"
-                    "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-                    "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-                    "mov.b32 %0, {b0, b1, b1, b1};\n\t}"
-                    : "=r"(b)
-                    : "f"(__uint_as_float(w[0] & 0x7FFFFFFFu) * mult),
-                      "f"(__uint_as_float(w[1] & 0x7FFFFFFFu) * mult),
-                      "f"(__uint_as_float(w[2] & 0x7FFFFFFFu) * mult),
-                      "f"(__uint_as_float(w[3] & 0x7FFFFFFFu) * mult));
-                c = (b & 0xFFFFu) | ((w[0] >> 28) & 0x8u) | ((w[1] >> 24) & 0x80u) |
-                    ((w[2] >> 20) & 0x800u) | ((w[3] >> 16) & 0x8000u);
-            }
-            s_codes[wid][32 * j + lane] = static_cast<uint16_t>(nf ? 0u : c);
-            if ((lane & 7) == 0)
-                s_scales[wid][4 * j + (lane >> 3)] = static_cast<uint8_t>(nf ? 0xFFu : s + 127);
+            uint32_t b;
+            asm("{\n\t.reg .b8 b0, b1;\n\t"
+                "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+                "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+                "mov.b32 %0, {b0, b1, b1, b1};\n\t}"
+                : "=r"(b)
+                : "f"(__uint_as_float(w[0] & 0x7FFFFFFFu) * mult),
+                  "f"(__uint_as_float(w[1] & 0x7FFFFFFFu) * mult),
+                  "f"(__uint_as_float(w[2] & 0x7FFFFFFFu) * mult),
+                  "f"(__uint_as_float(w[3] & 0x7FFFFFFFu) * mult));
+            const uint32_t cw = (b & 0xFFFFu) | ((w[0] >> 28) & 0x8u) | ((w[1] >> 24) & 0x80u) |
+                                ((w[2] >> 20) & 0x800u) | ((w[3] >> 16) & 0x8000u);
+            const uint32_t S = nf ? 0xFFu : static_cast<uint32_t>(s + 127);
+            const int64_t blk = blk0 + 4 * j + (lane >> 3);
+            if (blk < n_blocks)
+                __stcs(codes + blk0 * 8 + 32 * j + lane, static_cast<uint16_t>(nf ? 0u : cw));
+            // block 4j + q (q = 0..3) lives on lanes 8q .. 8q+7; lane 4j + q takes its scale
+            const uint32_t got = __shfl_sync(0xFFFFFFFFu, S, (lane & 3) * 8);
+            if ((lane >> 2) == j) mine = got;
         }
-        __syncwarp();
-        const int64_t blk = step * 32 + lane;
-        if (blk < n_blocks) {
-            codes[blk] = reinterpret_cast<const uint4*>(s_codes[wid])[lane];
-            scales[blk] = s_scales[wid][lane];
+        if (blk0 + lane < n_blocks) scales[blk0 + lane] = static_cast<uint8_t>(mine);
+        if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
         }
-        __syncwarp();
     }
 }
 
 // ---------------------------------------------------------------- MXFP4 -> bf16
-// One warp step = 128 chunks of 8 elements (4 code bytes -> 16 output bytes);
-// lane l handles chunks 32j + l so that every load and store is coalesced.
-__global__ void __launch_bounds__(kQThreads)
-dequantize_kernel(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                  int64_t n_chunks, uint4* __restrict__ out) {
-    const int lane = threadIdx.x & 31;
-    const int64_t n_steps = (n_chunks + 127) >> 7;
-    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t step = warp0; step < n_steps; step += nwarps) {
-        uint32_t cw[4], S[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t ch = step * 128 + 32 * j + lane;
-            cw[j] = ch < n_chunks ? __ldcs(codes + ch) : 0u;
-            S[j] = ch < n_chunks ? scales[ch >> 2] : 127u;
+// Chunk = 1024 blocks: 16 KB of codes and 1 KB of scales per stage.  Consumer
+// thread i expands code words i + 256 m (m = 0..15) of the chunk; the output of
+// a warp instruction is 512 contiguous bytes.  The last few scale bytes of a
+// ragged final chunk (fewer than 16) are read from global memory directly,
+// since a bulk copy moves whole 16-byte units.
+constexpr int kDqChunkBlocks = 1024;
+
+__global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
+dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                  int64_t n_blocks, uint4* __restrict__ out, unsigned* status) {
+    constexpr int kCodeBytes = kDqChunkBlocks * 16;
+    constexpr int kStageBytes = kCodeBytes + kDqChunkBlocks;
+    constexpr int kStages = kRingSmemBytes / kStageBytes;   // 5
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ Ring ring;
+    ring_init(ring, kStages);
+    const int warp = threadIdx.x >> 5;
+    const int64_t n_chunks = (n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks;
+    if (warp == kRingConsumerWarps) {
+        if ((threadIdx.x & 31) == 0)
+            ring_produce(ring, kStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
+                const int64_t nb = min(static_cast<int64_t>(kDqChunkBlocks), n_blocks - c * kDqChunkBlocks);
+                const uint32_t cb = static_cast<uint32_t>(nb * 16);
+                const uint32_t sb = static_cast<uint32_t>(nb & ~int64_t{15});
+                mbar_arrive_expect_tx(bar, cb + sb);
+                uint8_t* dst = smem + st * kStageBytes;
+                bulk_load(dst, codes + c * kCodeBytes, cb, bar);
+                if (sb) bulk_load(dst + kCodeBytes, scales + c * kDqChunkBlocks, sb, bar);
+            }, status);
+        return;
+    }
+    int st = 0;
+    uint32_t ph = 0;
+    const int tid = threadIdx.x;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        if (!ring_wait_full(ring, st, ph, status)) break;
+        const int64_t nb = min(static_cast<int64_t>(kDqChunkBlocks), n_blocks - c * kDqChunkBlocks);
+        const int nw = static_cast<int>(nb * 4);                 // code words in this chunk
+        const int sb = static_cast<int>(nb & ~int64_t{15});      // scales staged in shared memory
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(smem + st * kStageBytes);
+        const uint8_t* sc = smem + st * kStageBytes + kCodeBytes;
+        uint4* o = out + c * (kDqChunkBlocks * 4);
+#pragma unroll 4
+        for (int m = 0; m < 16; ++m) {
+            const int i = tid + 256 * m;
+            if (i < nw) {
+                const int b = i >> 2;
+                const uint32_t S = b < sb ? sc[b] : __ldg(scales + c * kDqChunkBlocks + b);
+                __stcs(o + i, dequant8(cw[i], S));
+            }
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t ch = step * 128 + 32 * j + lane;
-            if (ch < n_chunks) __stcs(out + ch, dequant8(cw[j], S[j]));
+        ring_release(ring, st);
+        if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
         }
     }
 }
 
-int grid_for(int64_t n_steps, int sm_count) {
-    const int64_t per_cta = kWarpsPerCta;
-    int64_t g = (n_steps + per_cta - 1) / per_cta;
-    const int64_t cap = static_cast<int64_t>(sm_count) * 8;   // 8 CTAs of 256 threads per SM
-    return static_cast<int>(g < cap ? (g < 1 ? 1 : g) : cap);
+int ring_grid(int64_t n_chunks, int sm_count) {
+    const int64_t cap = static_cast<int64_t>(sm_count) * kRingCtasPerSm;
+    return static_cast<int>(n_chunks < cap ? (n_chunks < 1 ? 1 : n_chunks) : cap);
+}
+
+// Opt the kernel in to the ring's dynamic shared memory (once per process; the
+// device is the same for every call of this library's process-wide cache).
+template <class K>
+cudaError_t set_ring_smem(K kern) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemBytes);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t cols,
                             uint8_t* codes, uint8_t* scales, int rule, int sm_count,
-                            cudaStream_t stream) {
+                            unsigned* status, cudaStream_t stream) {
     const int64_t n_blocks = rows * (cols / 32);
-    const int64_t n_steps = (n_blocks + 31) / 32;
-    const int grid = grid_for(n_steps, sm_count);
-    if (is_f32)
-        quantize_f32_kernel<<<grid, kQThreads, 0, stream>>>(
-            reinterpret_cast<const uint4*>(x), n_blocks, reinterpret_cast<uint4*>(codes), scales,
-            rule);
-    else
-        quantize_bf16_kernel<<<grid, kQThreads, 0, stream>>>(
-            reinterpret_cast<const uint4*>(x), n_blocks, reinterpret_cast<uint4*>(codes), scales,
-            rule, nullptr);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_qdq_bf16(const void* x, int64_t rows, int64_t cols, void* out, int sm_count,
-                            cudaStream_t stream) {
-    const int64_t n_blocks = rows * (cols / 32);
-    const int64_t n_steps = (n_blocks + 31) / 32;
-    quantize_bf16_kernel<<<grid_for(n_steps, sm_count), kQThreads, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), n_blocks, nullptr, nullptr, MXFP4_SCALE_FLOOR,
-        reinterpret_cast<uint4*>(out));
+    const int grid = ring_grid((n_blocks + kChunkBlocks - 1) / kChunkBlocks, sm_count);
+    cudaError_t e;
+    if (is_f32) {
+        if ((e = set_ring_smem(quantize_f32_kernel)) != cudaSuccess) return e;
+        quantize_f32_kernel<<<grid, kRingThreads, kRingSmemBytes, stream>>>(
+            static_cast<const uint8_t*>(x), n_blocks, reinterpret_cast<uint16_t*>(codes), scales,
+            rule, status);
+    } else {
+        if ((e = set_ring_smem(quantize_bf16_kernel)) != cudaSuccess) return e;
+        quantize_bf16_kernel<<<grid, kRingThreads, kRingSmemBytes, stream>>>(
+            static_cast<const uint8_t*>(x), n_blocks, reinterpret_cast<uint32_t*>(codes), scales,
+            rule, status);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
-                              int64_t cols, void* out, int sm_count, cudaStream_t stream) {
-    const int64_t n_chunks = rows * cols / 8;
-    const int64_t n_steps = (n_chunks + 127) / 128;
-    dequantize_kernel<<<grid_for(n_steps, sm_count), kQThreads, 0, stream>>>(
-        reinterpret_cast<const uint32_t*>(codes), scales, n_chunks, reinterpret_cast<uint4*>(out));
+                              int64_t cols, void* out, int sm_count, unsigned* status,
+                              cudaStream_t stream) {
+    const int64_t n_blocks = rows * (cols / 32);
+    const int grid = ring_grid((n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks, sm_count);
+    cudaError_t e = set_ring_smem(dequantize_kernel);
+    if (e != cudaSuccess) return e;
+    dequantize_kernel<<<grid, kRingThreads, kRingSmemBytes, stream>>>(
+        codes, scales, n_blocks, reinterpret_cast<uint4*>(out), status);
     return cudaGetLastError();
 }
 

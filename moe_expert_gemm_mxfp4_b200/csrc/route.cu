@@ -1,6 +1,6 @@
-// MoE routing for sm_100a: top-k + softmax, per-expert histogram with warp
-// ballots, prefix sums, the expert-sorted permutation of (token, slot) pairs,
-// the gather of token rows into that order, and the deterministic combine.
+// MoE routing for sm_100a: top-k + softmax, per-expert histogram, prefix sums,
+// the expert-sorted permutation of (token, slot) pairs, the gather of token rows
+// into that order, and the deterministic combine.
 //
 // The pages route MoE tokens through a downloadable MegaBlocks kernel and name
 // a top-k kernel (agentlenshq.com, "Transformers 4.40 performance upgrades for
@@ -8,23 +8,26 @@
 // rule itself is a reading: top-k by (logit desc, expert id asc), softmax over
 // the k selected logits, pairs p = t*k + j grouped by expert in ascending p.
 //
-// Kernels (one stream, no host synchronization):
-//   route_topk_count  per 64-token chunk: top-k/softmax (one warp per token),
-//                     then the chunk's per-expert counts and each pair's stable
-//                     rank inside the chunk (warp multisplit by ballots over the
-//                     bits of the expert id);
-//   route_scan        per expert: exclusive scan of the chunk counts; counts,
-//                     offsets (exclusive scan over experts);
-//   route_scatter     position of every pair, perm / inv / sorted weights, and
-//                     optionally the gather of its token row;
-//   moe_combine       out[t] = bf16(sum_j y[inv[t*k + j]]), fp32 rows summed in slot order.
+// Kernels (one stream, no host synchronization), sized for latency: every
+// token, expert and output vector gets its own warp or thread, so that a decode
+// step (tens of tokens) costs a few microseconds per launch.
+//   route_topk     one warp per token: top-k and softmax; per CTA (a chunk of
+//                  8 tokens) the per-expert pair counts and each pair's rank
+//                  among the chunk's pairs of its expert;
+//   route_scan     one CTA per expert: exclusive scan of its chunk counts ->
+//                  per-chunk base ranks, and the expert's total;
+//   route_scatter  offsets (exclusive scan over experts, recomputed per CTA in
+//                  shared memory), the position of every pair, perm / inv /
+//                  sorted weights, and optionally the gather of token rows;
+//   moe_combine    one thread per 8 output columns of a token:
+//                  out[t] = bf16(sum_j y[inv[t*k + j]]), fp32, slot order.
 #include "common.cuh"
 #include "internal.h"
 
 namespace mx {
 
-constexpr int kRouteTokPerCta = 64;
 constexpr int kRouteThreads = 256;
+constexpr int kTokPerChunk = kRouteThreads / 32;   // one warp per token
 constexpr int kMaxTopK = 8;
 constexpr int kMaxExperts = 256;
 
@@ -35,21 +38,15 @@ __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
 }
 
 __global__ void __launch_bounds__(kRouteThreads)
-route_topk_count_kernel(const float* __restrict__ logits, int T, int E, int k,
-                        int32_t* __restrict__ ids, float* __restrict__ weights,
-                        int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank) {
-    __shared__ int32_t s_ids[kRouteTokPerCta * kMaxTopK];
-    __shared__ int32_t s_seg[2 * (kRouteThreads / 32)][kMaxExperts];
+route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ ids,
+                  float* __restrict__ weights, int32_t* __restrict__ chunk_counts,
+                  int32_t* __restrict__ local_rank) {
+    __shared__ int32_t s_ids[kTokPerChunk * kMaxTopK];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int t0 = blockIdx.x * kRouteTokPerCta;
-    const int ntok = min(kRouteTokPerCta, T - t0);
-
-    for (int i = threadIdx.x; i < 2 * (kRouteThreads / 32) * kMaxExperts; i += blockDim.x)
-        (&s_seg[0][0])[i] = 0;
-
-    // ---- top-k + softmax, one warp per token
-    for (int lt = wid; lt < ntok; lt += kRouteThreads / 32) {
-        const int t = t0 + lt;
+    const int t0 = blockIdx.x * kTokPerChunk;
+    const int ntok = min(kTokPerChunk, T - t0);
+    const int t = t0 + wid;
+    if (wid < ntok) {
         float v[kMaxExperts / 32];
 #pragma unroll
         for (int i = 0; i < kMaxExperts / 32; ++i) {
@@ -59,132 +56,154 @@ route_topk_count_kernel(const float* __restrict__ logits, int T, int E, int k,
         uint32_t taken = 0;
         float sel_v[kMaxTopK];
         int sel_id[kMaxTopK];
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int bid = 0x7FFFFFFF;
 #pragma unroll
-            for (int i = 0; i < kMaxExperts / 32; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E && !((taken >> i) & 1u) && (bid == 0x7FFFFFFF || better(v[i], e, bv, bid))) {
-                    bv = v[i];
-                    bid = e;
-                }
-            }
+        for (int j = 0; j < kMaxTopK; ++j) {
+            sel_v[j] = -INFINITY;
+            sel_id[j] = 0;
+            if (j < k) {
+                float bv = -INFINITY;
+                int bid = 0x7FFFFFFF;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-                const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, o);
-                if (oid != 0x7FFFFFFF && (bid == 0x7FFFFFFF || better(ov, oid, bv, bid))) {
-                    bv = ov;
-                    bid = oid;
+                for (int i = 0; i < kMaxExperts / 32; ++i) {
+                    const int e = lane + 32 * i;
+                    if (e < E && !((taken >> i) & 1u) &&
+                        (bid == 0x7FFFFFFF || better(v[i], e, bv, bid))) {
+                        bv = v[i];
+                        bid = e;
+                    }
                 }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+                    const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, o);
+                    if (oid != 0x7FFFFFFF && (bid == 0x7FFFFFFF || better(ov, oid, bv, bid))) {
+                        bv = ov;
+                        bid = oid;
+                    }
+                }
+                if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
+                sel_v[j] = bv;   // uniform across the warp after the butterfly
+                sel_id[j] = bid;
             }
-            if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
-            sel_v[j] = bv;
-            sel_id[j] = bid;
         }
-        if (lane == 0) {
-            float z[kMaxTopK];
-            float sum = 0.f;
-            for (int j = 0; j < k; ++j) {
-                z[j] = expf(sel_v[j] - sel_v[0]);
-                sum += z[j];
+        // softmax over the k selected logits: lane j < k writes slot j
+        float sum = 0.f, mine = 0.f;
+        int my_id = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < k) {
+                const float z = expf(sel_v[j] - sel_v[0]);
+                sum += z;
+                if (lane == j) {
+                    mine = z;
+                    my_id = sel_id[j];
+                }
             }
-            for (int j = 0; j < k; ++j) {
-                ids[static_cast<int64_t>(t) * k + j] = sel_id[j];
-                weights[static_cast<int64_t>(t) * k + j] = z[j] / sum;
-                s_ids[lt * k + j] = sel_id[j];
-            }
+        }
+        if (lane < k) {
+            ids[static_cast<int64_t>(t) * k + lane] = my_id;
+            weights[static_cast<int64_t>(t) * k + lane] = mine / sum;
+            s_ids[wid * k + lane] = my_id;
         }
     }
     __syncthreads();
-
-    // ---- per-chunk histogram and stable ranks (warp multisplit by ballots)
+    // the chunk's pairs i = 0 .. ntok*k - 1 in ascending p: counts and stable ranks
     const int npairs = ntok * k;
-    int nbits = 0;
-    while ((1 << nbits) < E) ++nbits;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    int my_e[2], my_rank[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int i = r * kRouteThreads + threadIdx.x;
-        const bool valid = i < npairs;
-        const int e = valid ? s_ids[i] : 0;
-        uint32_t peers = __ballot_sync(0xFFFFFFFFu, valid);
-        for (int b = 0; b < nbits; ++b) {
-            const uint32_t bit = (e >> b) & 1;
-            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, bit);
-            peers &= bit ? bal : ~bal;
-        }
-        my_e[r] = e;
-        my_rank[r] = __popc(peers & lt_mask);
-        if (valid && (peers & lt_mask) == 0) s_seg[r * (kRouteThreads / 32) + wid][e] = __popc(peers);
+    if (static_cast<int>(threadIdx.x) < npairs) {
+        const int e = s_ids[threadIdx.x];
+        int r = 0;
+        for (int i = 0; i < static_cast<int>(threadIdx.x); ++i) r += s_ids[i] == e;
+        local_rank[static_cast<int64_t>(t0) * k + threadIdx.x] = r;
     }
-    __syncthreads();
-    const int nseg = 2 * (kRouteThreads / 32);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int sg = 0; sg < nseg; ++sg) {
-            const int c = s_seg[sg][e];
-            s_seg[sg][e] = run;
-            run += c;
-        }
-        chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = run;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int i = r * kRouteThreads + threadIdx.x;
-        if (i < npairs)
-            local_rank[static_cast<int64_t>(t0) * k + i] =
-                s_seg[r * (kRouteThreads / 32) + wid][my_e[r]] + my_rank[r];
+        int c = 0;
+        for (int i = 0; i < npairs; ++i) c += s_ids[i] == e;
+        chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = c;
     }
 }
 
-__global__ void __launch_bounds__(kMaxExperts)
-route_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
-                  int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
-    __shared__ int32_t s[kMaxExperts];
-    const int e = threadIdx.x;
-    int total = 0;
-    if (e < E) {
-        for (int c = 0; c < n_chunks; ++c) {
-            int32_t* p = chunk_counts + static_cast<int64_t>(c) * E + e;
-            const int v = *p;
-            *p = total;
-            total += v;
-        }
-        counts[e] = total;
+// Block-wide exclusive scan of one int per thread (blockDim.x == kRouteThreads);
+// returns the thread's exclusive prefix and sets *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
+    __shared__ int s_warp[kRouteThreads / 32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
     }
-    s[e] = e < E ? total : 0;
+    if (lane == 31) s_warp[wid] = x;
     __syncthreads();
-    for (int o = 1; o < kMaxExperts; o <<= 1) {     // inclusive Hillis-Steele scan
-        const int add = e >= o ? s[e - o] : 0;
-        __syncthreads();
-        s[e] += add;
-        __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kRouteThreads / 32; ++w) {
+        const int s = s_warp[w];
+        if (w < wid) base += s;
+        tot += s;
     }
-    if (e < E) offsets[e + 1] = s[e];
-    if (e == 0) offsets[0] = 0;
+    __syncthreads();   // s_warp may be reused by a later scan
+    *total = tot;
+    return base + x - v;
+}
+
+// One CTA per expert e: chunk_counts[c][e] <- exclusive prefix over chunks c;
+// counts[e] <- total.  Each thread scans a contiguous run of chunks.
+__global__ void __launch_bounds__(kRouteThreads)
+route_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
+                  int32_t* __restrict__ counts) {
+    const int e = blockIdx.x;
+    const int per = (n_chunks + kRouteThreads - 1) / kRouteThreads;
+    const int c0 = threadIdx.x * per;
+    const int c1 = min(n_chunks, c0 + per);
+    int run = 0;
+    for (int c = c0; c < c1; ++c) run += chunk_counts[static_cast<int64_t>(c) * E + e];
+    int total;
+    int base = block_exclusive_scan(run, &total);
+    for (int c = c0; c < c1; ++c) {
+        int32_t* p = chunk_counts + static_cast<int64_t>(c) * E + e;
+        const int v = *p;
+        *p = base;
+        base += v;
+    }
+    if (threadIdx.x == 0) counts[e] = total;
 }
 
 // One warp per pair: its sorted position, the routing tables and, if `x` is
-// given, the copy of its token's row into the expert-sorted activation matrix.
+// given, the copy of its token's row into the expert-sorted activation matrix
+// (row_vec 16-byte vectors per row); if `xs` is given, likewise for a second
+// matrix of xs_row bytes per row (the block scales of MXFP4 activations).
+// Every CTA first recomputes offsets (exclusive scan of counts over experts);
+// CTA 0 also stores them.
 __global__ void __launch_bounds__(kRouteThreads)
 route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ weights,
                      const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ local_rank,
-                     const int32_t* __restrict__ offsets, int64_t P, int k, int E,
-                     int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                     const int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int64_t P,
+                     int k, int E, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                      float* __restrict__ w_sorted, const uint4* __restrict__ x, int64_t row_vec,
-                     uint4* __restrict__ x_sorted) {
+                     uint4* __restrict__ x_sorted, const uint8_t* __restrict__ xs, int64_t xs_row,
+                     uint8_t* __restrict__ xs_sorted) {
+    __shared__ int32_t s_off[kMaxExperts];
+    {
+        const int e = threadIdx.x;   // E <= kMaxExperts == blockDim.x
+        const int c = e < E ? counts[e] : 0;
+        int total;
+        const int ex = block_exclusive_scan(c, &total);
+        if (e < E) s_off[e] = ex;
+        if (blockIdx.x == 0) {
+            if (e < E) offsets[e] = ex;
+            if (e == 0) offsets[E] = total;
+        }
+        __syncthreads();
+    }
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t p = warp0; p < P; p += nwarps) {
         const int e = ids[p];
         const int64_t t = p / k;
-        const int64_t chunk = t / kRouteTokPerCta;
-        const int64_t pos = static_cast<int64_t>(offsets[e]) + chunk_base[chunk * E + e] + local_rank[p];
+        const int64_t chunk = t / kTokPerChunk;
+        const int64_t pos = static_cast<int64_t>(s_off[e]) + chunk_base[chunk * E + e] + local_rank[p];
         if (lane == 0) {
             perm[pos] = static_cast<int32_t>(p);
             inv[p] = static_cast<int32_t>(pos);
@@ -195,6 +214,11 @@ route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
             uint4* dst = x_sorted + pos * row_vec;
             for (int64_t c = lane; c < row_vec; c += 32) dst[c] = __ldg(src + c);
         }
+        if (xs) {
+            const uint8_t* src = xs + t * xs_row;
+            uint8_t* dst = xs_sorted + pos * xs_row;
+            for (int64_t c = lane; c < xs_row; c += 32) dst[c] = __ldg(src + c);
+        }
     }
 }
 
@@ -203,69 +227,72 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// One warp per token; its k fp32 rows are summed in slot order j = 0..k-1 and
-// rounded once to bf16.
+// One thread per 8 output columns of one token; the token's k fp32 rows are
+// summed in slot order j = 0..k-1 and rounded once to bf16.
 __global__ void __launch_bounds__(kRouteThreads)
 moe_combine_kernel(const float4* __restrict__ y_sorted, const int32_t* __restrict__ inv,
                    int64_t T, int k, int64_t row_vec8, uint4* __restrict__ out) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t t = warp0; t < T; t += nwarps) {
-        int64_t rows[kMaxTopK];
-        for (int j = 0; j < k; ++j) rows[j] = inv[t * k + j];
-        for (int64_t c = lane; c < row_vec8; c += 32) {
-            float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int j = 0; j < k; ++j) {
-                const float4* src = y_sorted + (rows[j] * row_vec8 + c) * 2;
+    const int64_t n = T * row_vec8;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const int64_t t = i / row_vec8, c = i - t * row_vec8;
+        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < k) {
+                const int64_t row = __ldg(inv + t * k + j);
+                const float4* src = y_sorted + (row * row_vec8 + c) * 2;
                 const float4 u = __ldcs(src), v = __ldcs(src + 1);
                 a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
                 a[4] += v.x; a[5] += v.y; a[6] += v.z; a[7] += v.w;
             }
-            uint4 o;
-            o.x = pack_bf16x2(a[0], a[1]);
-            o.y = pack_bf16x2(a[2], a[3]);
-            o.z = pack_bf16x2(a[4], a[5]);
-            o.w = pack_bf16x2(a[6], a[7]);
-            out[t * row_vec8 + c] = o;
         }
+        uint4 o;
+        o.x = pack_bf16x2(a[0], a[1]);
+        o.y = pack_bf16x2(a[2], a[3]);
+        o.z = pack_bf16x2(a[4], a[5]);
+        o.w = pack_bf16x2(a[6], a[7]);
+        out[i] = o;
     }
 }
 
 }  // namespace
 
 size_t route_tmp_bytes(int64_t T, int64_t E, int top_k) {
-    const int64_t n_chunks = (T + kRouteTokPerCta - 1) / kRouteTokPerCta;
+    const int64_t n_chunks = (T + kTokPerChunk - 1) / kTokPerChunk;
     return static_cast<size_t>(n_chunks * E + T * top_k) * sizeof(int32_t);
 }
 
 cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, int32_t* ids,
                          float* weights, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv, float* w_sorted, void* tmp, const void* x, int64_t H,
-                         void* x_sorted, int sm_count, cudaStream_t stream) {
-    const int64_t n_chunks = (T + kRouteTokPerCta - 1) / kRouteTokPerCta;
+                         int32_t* inv, float* w_sorted, void* tmp, const void* x,
+                         int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
+                         void* xs_sorted, int sm_count, cudaStream_t stream) {
+    const int64_t n_chunks = (T + kTokPerChunk - 1) / kTokPerChunk;
     int32_t* chunk_counts = static_cast<int32_t*>(tmp);
     int32_t* local_rank = chunk_counts + n_chunks * E;
-    route_topk_count_kernel<<<static_cast<unsigned>(n_chunks), kRouteThreads, 0, stream>>>(
+    route_topk_kernel<<<static_cast<unsigned>(n_chunks), kRouteThreads, 0, stream>>>(
         logits, static_cast<int>(T), static_cast<int>(E), top_k, ids, weights, chunk_counts,
         local_rank);
-    route_scan_kernel<<<1, kMaxExperts, 0, stream>>>(chunk_counts, static_cast<int>(n_chunks),
-                                                     static_cast<int>(E), counts, offsets);
+    route_scan_kernel<<<static_cast<unsigned>(E), kRouteThreads, 0, stream>>>(
+        chunk_counts, static_cast<int>(n_chunks), static_cast<int>(E), counts);
     const int64_t P = T * top_k;
-    const int64_t warps_needed = P;
-    int64_t grid = (warps_needed + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
+    int64_t grid = (P + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
     const int64_t cap = static_cast<int64_t>(sm_count) * 8;
     if (grid > cap) grid = cap;
     route_scatter_kernel<<<static_cast<unsigned>(grid), kRouteThreads, 0, stream>>>(
-        ids, weights, chunk_counts, local_rank, offsets, P, top_k, static_cast<int>(E), perm, inv,
-        w_sorted, static_cast<const uint4*>(x), H / 8, static_cast<uint4*>(x_sorted));
+        ids, weights, chunk_counts, local_rank, counts, offsets, P, top_k, static_cast<int>(E),
+        perm, inv, w_sorted, static_cast<const uint4*>(x), row_bytes / 16,
+        static_cast<uint4*>(x_sorted), static_cast<const uint8_t*>(xs), xs_row_bytes,
+        static_cast<uint8_t*>(xs_sorted));
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, int top_k,
                            int64_t H, void* out, int sm_count, cudaStream_t stream) {
-    int64_t grid = (T + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
-    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    const int64_t n = T * (H / 8);
+    int64_t grid = (n + kRouteThreads - 1) / kRouteThreads;
+    const int64_t cap = static_cast<int64_t>(sm_count) * 16;
     if (grid > cap) grid = cap;
     moe_combine_kernel<<<static_cast<unsigned>(grid), kRouteThreads, 0, stream>>>(
         static_cast<const float4*>(y_sorted), inv, T, top_k, H / 8, static_cast<uint4*>(out));

@@ -87,7 +87,9 @@ def test_gemm_extreme_scales_use_exact_path():
         assert np.array_equal(got[m], deq[:, m * 4])
 
 
-@pytest.mark.parametrize("M,K,N", [(8, 256, 512), (33, 448, 130), (300, 1024, 512)])
+@pytest.mark.parametrize("M,K,N", [(1, 64, 1), (8, 256, 512), (16, 128, 128), (17, 192, 200),
+                                   (33, 448, 130), (64, 320, 384), (300, 1024, 512),
+                                   (257, 704, 640), (1024, 2880, 2880)])
 def test_gemm_w4a4(M, K, N):
     g = torch.Generator().manual_seed(M + K + N + 1)
     x = torch.randn(M, K, generator=g).to(torch.bfloat16)
@@ -95,3 +97,39 @@ def test_gemm_w4a4(M, K, N):
     wc, ws = oracle_quantize_weights(w)
     y = _run(x, wc, ws, mx.W4A4)
     assert_close_tol(y, oracle.gemm_w4a4(bits_of(x), wc, ws), what=f"w4a4 {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("M", [5, 40, 100, 200])
+def test_gemm_w4a4_one_hot_selects_weight_column(M):
+    """x rows with a single 1.0 are on the MXFP4 grid (block scale 2^-2, code 4):
+    every output is one product of block-scaled E2M1 values, so y[m] equals the
+    bf16 of dequantized weight column k exactly; a misplaced weight or activation
+    block scale shows up as a power-of-two error."""
+    K, N = 512, 300
+    g = torch.Generator().manual_seed(40 + M)
+    w = torch.randn(N, K, generator=g) * 0.05
+    wc, ws = oracle_quantize_weights(w)
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    for m in range(M):
+        x[m, (m * 37) % K] = 1.0
+    y = _run(x, wc, ws, mx.W4A4)
+    W = oracle.dequantize_f64(wc, ws)
+    for m in range(M):
+        col = W[:, (m * 37) % K]
+        assert np.array_equal(y[m], oracle.bf16_to_f64(oracle.f64_to_bf16(col))), m
+
+
+def test_gemm_w4a4_equals_w4a16_on_grid_activations():
+    """Activations already on the MXFP4 grid (dequantized random codes) quantize to
+    themselves, so W4A4 and W4A16 compute the same products; they differ only in
+    fp32 summation order."""
+    M, K, N = 96, 768, 384
+    g = torch.Generator().manual_seed(11)
+    xc = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8).numpy()
+    xs = torch.randint(118, 130, (M, K // 32), generator=g, dtype=torch.uint8).numpy()
+    x = torch.from_numpy(oracle.dequantize_bf16(xc, xs).view(np.int16)).view(torch.bfloat16)
+    w = torch.randn(N, K, generator=g) * 0.05
+    wc, ws = oracle_quantize_weights(w)
+    y4 = _run(x, wc, ws, mx.W4A4)
+    y16 = _run(x, wc, ws, mx.W4A16)
+    assert_close_tol(y4, y16, what="w4a4 vs w4a16 on grid")
