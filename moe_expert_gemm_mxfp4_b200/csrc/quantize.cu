@@ -66,7 +66,9 @@ __device__ __forceinline__ float inv_pow2(int s) {
     return __uint_as_float(static_cast<uint32_t>(127 - s) << 23);
 }
 
-// 8 magnitudes (already scaled) -> 4 packed E2M1 bytes; element 2i in the low nibble.
+// 8 values (already scaled, signed) -> 4 packed E2M1 bytes; element 2i in the low
+// nibble.  The conversion rounds to nearest even, saturates at 6 and keeps the sign
+// of its input, zero results included (-0 and small negatives give code 8).
 __device__ __forceinline__ uint32_t cvt_e2m1x8(float e0, float e1, float e2, float e3, float e4,
                                                float e5, float e6, float e7) {
     uint32_t out;
@@ -81,36 +83,31 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float e0, float e1, float e2, flo
     return out;
 }
 
-__device__ __forceinline__ float bf16_mag(uint32_t h16) {
-    return __uint_as_float((h16 & 0x7FFFu) << 16);
-}
+// The two bf16 halves of a word as fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Sign bits of the two bf16 halves of w at bits 3 and 7 of a code byte.
-__device__ __forceinline__ uint32_t bf16x2_sign_nibbles(uint32_t w) {
-    return ((w >> 12) & 0x8u) | ((w >> 24) & 0x80u);
-}
-
-// 8 bf16 elements (one uint4) -> 4 code bytes given the block multiplier 2^-s.
+// 8 bf16 elements (one uint4) -> 4 code bytes given the block multiplier 2^-s
+// (an exact power-of-two product in fp32).
 __device__ __forceinline__ uint32_t quant8_bf16(uint4 v, float mult) {
-    uint32_t c = cvt_e2m1x8(bf16_mag(v.x) * mult, bf16_mag(v.x >> 16) * mult,
-                            bf16_mag(v.y) * mult, bf16_mag(v.y >> 16) * mult,
-                            bf16_mag(v.z) * mult, bf16_mag(v.z >> 16) * mult,
-                            bf16_mag(v.w) * mult, bf16_mag(v.w >> 16) * mult);
-    c |= bf16x2_sign_nibbles(v.x) | (bf16x2_sign_nibbles(v.y) << 8) |
-         (bf16x2_sign_nibbles(v.z) << 16) | (bf16x2_sign_nibbles(v.w) << 24);
-    return c;
+    return cvt_e2m1x8(bf16_lo(v.x) * mult, bf16_hi(v.x) * mult, bf16_lo(v.y) * mult,
+                      bf16_hi(v.y) * mult, bf16_lo(v.z) * mult, bf16_hi(v.z) * mult,
+                      bf16_lo(v.w) * mult, bf16_hi(v.w) * mult);
 }
 
-__device__ __forceinline__ uint32_t amax8_bf16(uint4 v, uint32_t& nonfinite) {
-    uint32_t m = 0;
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = w[i] & 0x7FFFu, hi = (w[i] >> 16) & 0x7FFFu;
-        nonfinite |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
-        m = max(m, max(lo, hi));
-    }
-    return m;
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Largest magnitude bit pattern (15 bits) of 8 bf16 elements.  As unsigned
+// integers, magnitudes order like the values; Inf and NaN (0x7F80 and above)
+// order above every finite value, so a block is non-finite iff its amax >= 0x7F80.
+__device__ __forceinline__ uint32_t amax8_bf16(uint4 v) {
+    const uint32_t m = max_u16x2(max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                 max_u16x2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
 }
 
 // Dequantize 8 codes (one 32-bit code word) with the block's scale byte -> 8 bf16.
@@ -121,6 +118,34 @@ __device__ __forceinline__ uint4 dequant8(uint32_t cw, uint32_t S) {
     o.y = dequant_byte_exact((cw >> 8) & 0xFFu, sc);
     o.z = dequant_byte_exact((cw >> 16) & 0xFFu, sc);
     o.w = dequant_byte_exact(cw >> 24, sc);
+    return o;
+}
+
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+// Dequantize one code word through the lane-replicated LUT of bf16 pairs (entry
+// (b, lane) at lut + b * 256 + lane * 4): for S in [2, 254] the LUT value times
+// 2^(S-127) is one exact bf16x2 product (normal operands; a product past the
+// bf16 range rounds to Inf as round-to-nearest-even does).  S in {0, 1, 255} takes
+// the exact fp32 route.
+__device__ __forceinline__ uint4 dequant8_lut(uint32_t cw, uint32_t S, uint32_t lut_lane) {
+    if (S - 2u > 252u) return dequant8(cw, S);
+    const uint32_t sf = S * 0x00800080u;   // bf16x2 {2^(S-127), 2^(S-127)}
+    uint4 o;
+    o.x = bmul2(lds32(prmt(cw, 0u, 0x4404u) + lut_lane), sf);
+    o.y = bmul2(lds32(prmt(cw, 0u, 0x4414u) + lut_lane), sf);
+    o.z = bmul2(lds32(prmt(cw, 0u, 0x4424u) + lut_lane), sf);
+    o.w = bmul2(lds32(prmt(cw, 0u, 0x4434u) + lut_lane), sf);
     return o;
 }
 
@@ -139,11 +164,11 @@ struct Ring {
     int abort;
 };
 
-__device__ __forceinline__ void ring_init(Ring& r, int n_stages) {
+__device__ __forceinline__ void ring_init(Ring& r, int n_stages, int consumer_warps = kRingConsumerWarps) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < n_stages; ++i) {
             mbar_init(&r.full[i], 1);
-            mbar_init(&r.empty[i], kRingConsumerWarps);
+            mbar_init(&r.empty[i], consumer_warps);
         }
         r.abort = 0;
         fence_mbar_init();
@@ -238,12 +263,10 @@ quantize_bf16_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint32_t* 
         uint32_t mine = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            uint32_t nf = 0;
-            uint32_t am = amax8_bf16(v[j], nf);
+            uint32_t am = amax8_bf16(v[j]);
             am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
             am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
-            nf |= __shfl_xor_sync(0xFFFFFFFFu, nf, 1);
-            nf |= __shfl_xor_sync(0xFFFFFFFFu, nf, 2);
+            const bool nf = am >= 0x7F80u;
             const int s = block_exp_bf16(am, rule);
             const uint32_t cw = nf ? 0u : quant8_bf16(v[j], inv_pow2(s));
             const uint32_t S = nf ? 0xFFu : static_cast<uint32_t>(s + 127);
@@ -298,33 +321,23 @@ quantize_f32_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint16_t* _
         uint32_t mine = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-            uint32_t am = 0, nf = 0;
+            // magnitudes order like unsigned integers; Inf/NaN (>= 0x7F800000) above all
+            uint32_t am = max(max(v[j].x & 0x7FFFFFFFu, v[j].y & 0x7FFFFFFFu),
+                              max(v[j].z & 0x7FFFFFFFu, v[j].w & 0x7FFFFFFFu));
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t m = w[i] & 0x7FFFFFFFu;
-                nf |= (m & 0x7F800000u) == 0x7F800000u;
-                am = max(am, m);
-            }
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) {
-                am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-                nf |= __shfl_xor_sync(0xFFFFFFFFu, nf, o);
-            }
+            for (int o = 1; o < 8; o <<= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+            const bool nf = am >= 0x7F800000u;
             const int s = block_exp_f32(am, rule);
             const float mult = inv_pow2(s);
-            uint32_t b;
+            uint32_t cw;
             asm("{\n\t.reg .b8 b0, b1;\n\t"
                 "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
                 "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
                 "mov.b32 %0, {b0, b1, b1, b1};\n\t}"
-                : "=r"(b)
-                : "f"(__uint_as_float(w[0] & 0x7FFFFFFFu) * mult),
-                  "f"(__uint_as_float(w[1] & 0x7FFFFFFFu) * mult),
-                  "f"(__uint_as_float(w[2] & 0x7FFFFFFFu) * mult),
-                  "f"(__uint_as_float(w[3] & 0x7FFFFFFFu) * mult));
-            const uint32_t cw = (b & 0xFFFFu) | ((w[0] >> 28) & 0x8u) | ((w[1] >> 24) & 0x80u) |
-                                ((w[2] >> 20) & 0x800u) | ((w[3] >> 16) & 0x8000u);
+                : "=r"(cw)
+                : "f"(__uint_as_float(v[j].x) * mult), "f"(__uint_as_float(v[j].y) * mult),
+                  "f"(__uint_as_float(v[j].z) * mult), "f"(__uint_as_float(v[j].w) * mult));
+            cw &= 0xFFFFu;
             const uint32_t S = nf ? 0xFFu : static_cast<uint32_t>(s + 127);
             const int64_t blk = blk0 + 4 * j + (lane >> 3);
             if (blk < n_blocks)
@@ -342,59 +355,75 @@ quantize_f32_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint16_t* _
 }
 
 // ---------------------------------------------------------------- MXFP4 -> bf16
-// Chunk = 1024 blocks: 16 KB of codes and 1 KB of scales per stage.  Consumer
-// thread i expands code words i + 256 m (m = 0..15) of the chunk; the output of
-// a warp instruction is 512 contiguous bytes.  The last few scale bytes of a
-// ragged final chunk (fewer than 16) are read from global memory directly,
-// since a bulk copy moves whole 16-byte units.
+// Chunk = 1024 blocks: 16 KB of codes and 1 KB of scales per stage.  One CTA per
+// SM with 16 consumer warps and the 64 KB lane-replicated LUT of bf16 pairs
+// (dequant8_lut); consumer thread i expands code words i + 512 m (m = 0..7) of the
+// chunk, so a warp's output is 512 contiguous bytes per store instruction.  The
+// last few scale bytes of a ragged final chunk (fewer than 16) are read from
+// global memory directly, since a bulk copy moves whole 16-byte units.
 constexpr int kDqChunkBlocks = 1024;
+constexpr int kDqWarps = 16;
+constexpr int kDqThreads = (kDqWarps + 1) * 32;
+constexpr int kDqLutBytes = 256 * 256;
+constexpr int kDqStages = 8;
+constexpr int kDqCodeBytes = kDqChunkBlocks * 16;
+constexpr int kDqStageBytes = kDqCodeBytes + kDqChunkBlocks;
+constexpr int kDqSmemBytes = kDqLutBytes + kDqStages * kDqStageBytes;
 
-__global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
+__global__ void __launch_bounds__(kDqThreads, 1)
 dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                   int64_t n_blocks, uint4* __restrict__ out, unsigned* status) {
-    constexpr int kCodeBytes = kDqChunkBlocks * 16;
-    constexpr int kStageBytes = kCodeBytes + kDqChunkBlocks;
-    constexpr int kStages = kRingSmemBytes / kStageBytes;   // 5
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ Ring ring;
-    ring_init(ring, kStages);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
+    uint8_t* stages = smem + kDqLutBytes;
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+        const uint32_t b = static_cast<uint32_t>(i >> 5);
+        lut[(b << 6) | (i & 31)] = e2m1_bf16(b & 15u) | (e2m1_bf16(b >> 4) << 16);
+    }
+    ring_init(ring, kDqStages, kDqWarps);   // its __syncthreads also publishes the LUT
     const int warp = threadIdx.x >> 5;
     const int64_t n_chunks = (n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks;
-    if (warp == kRingConsumerWarps) {
+    if (warp == kDqWarps) {
         if ((threadIdx.x & 31) == 0)
-            ring_produce(ring, kStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
+            ring_produce(ring, kDqStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
                 const int64_t nb = min(static_cast<int64_t>(kDqChunkBlocks), n_blocks - c * kDqChunkBlocks);
                 const uint32_t cb = static_cast<uint32_t>(nb * 16);
                 const uint32_t sb = static_cast<uint32_t>(nb & ~int64_t{15});
                 mbar_arrive_expect_tx(bar, cb + sb);
-                uint8_t* dst = smem + st * kStageBytes;
-                bulk_load(dst, codes + c * kCodeBytes, cb, bar);
-                if (sb) bulk_load(dst + kCodeBytes, scales + c * kDqChunkBlocks, sb, bar);
+                uint8_t* dst = stages + st * kDqStageBytes;
+                bulk_load(dst, codes + c * kDqCodeBytes, cb, bar);
+                if (sb) bulk_load(dst + kDqCodeBytes, scales + c * kDqChunkBlocks, sb, bar);
             }, status);
         return;
     }
     int st = 0;
     uint32_t ph = 0;
     const int tid = threadIdx.x;
+    const uint32_t lut_lane = smem_u32(lut) + (threadIdx.x & 31) * 4;
     for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
         if (!ring_wait_full(ring, st, ph, status)) break;
         const int64_t nb = min(static_cast<int64_t>(kDqChunkBlocks), n_blocks - c * kDqChunkBlocks);
         const int nw = static_cast<int>(nb * 4);                 // code words in this chunk
         const int sb = static_cast<int>(nb & ~int64_t{15});      // scales staged in shared memory
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(smem + st * kStageBytes);
-        const uint8_t* sc = smem + st * kStageBytes + kCodeBytes;
-        uint4* o = out + c * (kDqChunkBlocks * 4);
-#pragma unroll 4
-        for (int m = 0; m < 16; ++m) {
-            const int i = tid + 256 * m;
-            if (i < nw) {
-                const int b = i >> 2;
-                const uint32_t S = b < sb ? sc[b] : __ldg(scales + c * kDqChunkBlocks + b);
-                __stcs(o + i, dequant8(cw[i], S));
-            }
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(stages + st * kDqStageBytes);
+        const uint8_t* sc = stages + st * kDqStageBytes + kDqCodeBytes;
+        uint32_t w[8], S[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int i = tid + 32 * kDqWarps * m;
+            const int b = i >> 2;
+            w[m] = i < nw ? cw[i] : 0u;
+            S[m] = i < nw ? (b < sb ? sc[b] : __ldg(scales + c * kDqChunkBlocks + b)) : 127u;
         }
         ring_release(ring, st);
-        if (++st == kStages) {
+        uint4* o = out + c * (kDqChunkBlocks * 4);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int i = tid + 32 * kDqWarps * m;
+            if (i < nw) __stcs(o + i, dequant8_lut(w[m], S[m], lut_lane));
+        }
+        if (++st == kDqStages) {
             st = 0;
             ph ^= 1u;
         }
@@ -439,10 +468,12 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int64
                               int64_t cols, void* out, int sm_count, unsigned* status,
                               cudaStream_t stream) {
     const int64_t n_blocks = rows * (cols / 32);
-    const int grid = ring_grid((n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks, sm_count);
-    cudaError_t e = set_ring_smem(dequantize_kernel);
+    const int64_t n_chunks = (n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks;
+    const int grid = static_cast<int>(n_chunks < sm_count ? n_chunks : sm_count);
+    cudaError_t e = cudaFuncSetAttribute(dequantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDqSmemBytes);
     if (e != cudaSuccess) return e;
-    dequantize_kernel<<<grid, kRingThreads, kRingSmemBytes, stream>>>(
+    dequantize_kernel<<<grid, kDqThreads, kDqSmemBytes, stream>>>(
         codes, scales, n_blocks, reinterpret_cast<uint4*>(out), status);
     return cudaGetLastError();
 }
