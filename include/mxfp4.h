@@ -93,7 +93,7 @@ MXFP4_API mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* sca
 /* ---------------------------------------------------------------- GEMM
  * y [M, N] bf16 = x [M, K] bf16 . dequant(W)^T, W = MXFP4 codes [N, K/2] +
  * scales [N, K/32]; fp32 accumulation, one rounding to bf16 at the end.
- * Requires K % 64 == 0 and K <= 8064 (the block scales of a 128-row weight tile
+ * Requires K % 64 == 0 and K <= 7680 (the block scales of a 128-row weight tile
  * are staged whole in shared memory); any M >= 1, N >= 1.  Workspace: W4A16 needs none
  * (ws may be NULL); W4A4 needs mxfp4_gemm_workspace_size() bytes (x quantized to
  * MXFP4: codes and block scales). */
@@ -129,7 +129,7 @@ MXFP4_API size_t moe_mxfp4_route_workspace_size(int64_t T, int64_t E, int32_t to
  *   out[t] = bf16( sum_j y_tj ) in slot order (deterministic; no atomics).
  * x bf16 [T, H]; router_logits fp32 [T, E]; w13 codes uint8 [E, 2I, H/2] +
  * scales uint8 [E, 2I, H/32]; w2 codes uint8 [E, H, I/2] + scales [E, H, I/32];
- * out bf16 [T, H].  Requires H % 64 == 0, I % 64 == 0, H, I <= 8064, 1 <= top_k <= min(E, 8),
+ * out bf16 [T, H].  Requires H % 64 == 0, I % 64 == 0, H, I <= 7680, 1 <= top_k <= min(E, 8),
  * E <= 256, T*top_k < 2^31.  ws must hold moe_mxfp4_workspace_size() bytes
  * (routing tables and the per-pair activations h / y). */
 MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,

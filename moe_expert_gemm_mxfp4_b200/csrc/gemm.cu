@@ -17,23 +17,27 @@
 //
 // Data flow (one persistent CTA per SM, 16 warps):
 //   warp 0        codes producer: per tile the block scales of its 128 rows
-//                 (bulk copy, double-buffered); per K stage the packed codes
-//                 (32 B per row, 32B-swizzled) -> a deep codes ring that the
-//                 dequant warps release as soon as they have read it.
+//                 (bulk copy, double-buffered); per group of four K stages the
+//                 packed codes (128 B per row, 128B-swizzled: rows this wide
+//                 stream from HBM at full rate) -> a codes ring that the dequant
+//                 warps release as soon as they have read it.
 //   warp 2        activation producer: per K stage TT bf16 tiles [NT x 64]
 //                 (128B-swizzled, the UMMA K-major layout) -> activation ring,
 //                 released by the MMA.
 //   warps 4..11   two dequant warpgroups (alternate stages): one weight row per
 //                 thread; codes -> bf16 through a lane-replicated 256-entry
-//                 shared LUT times the block scale 2^(S-127) (exact bf16
-//                 product), stored with tcgen05.st into TMEM: the dequantized
-//                 weights are the MMA's A operand and never touch shared memory.
+//                 shared LUT (one prmt forms an entry's address) times the block
+//                 scale 2^(S-127) (exact bf16 product), stored with tcgen05.st
+//                 into TMEM: the dequantized weights are the MMA's A operand and
+//                 never touch shared memory.
 //   warp 1        MMA issuer: tcgen05.mma kind::f16, M = 128, N = NT, K = 16,
 //                 A from TMEM, B from shared memory, D (fp32) in TMEM.
 //   warps 12..15  epilogue: tcgen05.ld of the accumulators, fused epilogue,
 //                 stores.
+// The MMA issuer waits once per group of four K stages: a wait between tcgen05
+// operations costs the issuing thread about the latency of the MMAs in flight.
 // TMEM: columns [0, 256) accumulators (TT*NT columns per buffer, double-buffered
-// when they fit), [256, 512) eight 32-column A slots.
+// when they fit), [256, 512) eight 32-column A slots (two sets of four).
 // Every mbarrier wait is time-bounded (MXFP4_ERR_TIMEOUT in the status word).
 #include "gemm_common.cuh"
 
@@ -51,7 +55,6 @@ constexpr int kSub = 4;             // 64-wide K sub-stages per codes super-stag
 constexpr int kCodeRowBytes = kSub * kBK / 2;          // 128 B of codes per weight row
 constexpr int kCodeBytes = kBM * kCodeRowBytes;        // one codes super-stage (16 KB)
 constexpr int kLutBytes = 256 * 256;   // 256 byte values x 256-B rows (32 lanes x bf16x2 used)
-constexpr int kXbufBytes = 0;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxRing = 16;
 constexpr int kMaxCodeStages = 4;
@@ -76,26 +79,49 @@ struct Cfg {
     static_assert(kAccCols <= kACol0, "accumulators overlap the A slots");
 };
 
-// Shared-memory layout, identical on host (sizing) and device.
+// Shared-memory layout, identical on host (sizing) and device.  Offsets count from
+// the start of dynamic shared memory, whose shared-window address is 1024 (the
+// window's first 1 KB is reserved and the kernel has no static shared memory; the
+// kernel checks this).  The dequant LUT sits at window address 64 KB, so that the
+// low 16 bits of an entry address are (code byte << 8) | (lane * 4) and one prmt
+// builds it.  Below the LUT: barriers, tile tables, the tile scales and as many
+// codes stages as fit; above it: the activation stages, then anything left over.
+constexpr int kWindowBase = 1024;
+constexpr int kLutOff = 65536 - kWindowBase;
+
 struct Layout {
-    int codes_off, acts_off, scales_off, scale_bytes, xbuf_off, bar_off, tstart_off, off_off,
-        misc_off, total;
+    int scales_off, scale_bytes, bar_off, tstart_off, off_off, misc_off;
+    int n_codes_lo, codes_lo_off, acts_off, codes_hi_off, total;
 };
 
 __host__ __device__ inline Layout make_layout(int act_stage_bytes, int code_stages, int act_stages,
                                               int K) {
     Layout L;
-    L.codes_off = kLutBytes;
-    L.acts_off = L.codes_off + code_stages * kCodeBytes;
-    L.scales_off = L.acts_off + act_stages * act_stage_bytes;
-    L.scale_bytes = ((kBM * (K / 32)) + 127) / 128 * 128;
-    L.xbuf_off = L.scales_off + 2 * L.scale_bytes;
-    L.bar_off = L.xbuf_off + kXbufBytes;
     const int n_bars = 4 * kMaxRing + 2 * kASlots + 2 + 2 + 2 + 2 + 1;
+    L.bar_off = 0;
     L.tstart_off = L.bar_off + n_bars * 8;
     L.off_off = L.tstart_off + (kMaxGroups + 1) * 4;
     L.misc_off = L.off_off + (kMaxGroups + 1) * 4;
-    L.total = L.misc_off + 16 + 1024;   // + slack for the 1024-B alignment of the base
+    int lo = (L.misc_off + 16 + 127) / 128 * 128;
+    int hi = kLutOff + kLutBytes;
+    L.acts_off = hi;
+    hi += act_stages * act_stage_bytes;
+    L.scale_bytes = ((kBM * (K / 32)) + 127) / 128 * 128;
+    if (lo + 2 * L.scale_bytes <= kLutOff) {
+        L.scales_off = lo;
+        lo += 2 * L.scale_bytes;
+    } else {
+        L.scales_off = hi;
+        hi += 2 * L.scale_bytes;
+    }
+    lo = (lo + 1023) / 1024 * 1024;
+    L.codes_lo_off = lo;
+    L.n_codes_lo = lo < kLutOff ? (kLutOff - lo) / kCodeBytes : 0;
+    if (L.n_codes_lo > code_stages) L.n_codes_lo = code_stages;
+    hi = (hi + 1023) / 1024 * 1024;
+    L.codes_hi_off = hi;
+    hi += (code_stages - L.n_codes_lo) * kCodeBytes;
+    L.total = hi;
     return L;
 }
 
@@ -116,10 +142,10 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 // exact because both factors and the product are normal bf16 numbers (or the
 // product overflows to Inf, as round-to-nearest-even does).  Otherwise the
 // exact fp32 route (subnormal results for S <= 1, NaN for S = 255).
-// LUT entry (b, lane) sits at lut_base + b * 256 + lane * 4 (lane-replicated, so
-// the 32 lanes of a warp hit 32 different banks whatever their bytes); lut_lane
-// is lut_base + lane * 4 and one prmt places code byte j of a word at bits 8..15,
-// which makes the row address b * 256 without a multiply.
+// LUT entry (b, lane) sits at window address 65536 + b * 256 + lane * 4 (lane-
+// replicated, so the 32 lanes of a warp hit 32 different banks whatever their
+// bytes); lut_lane = 65536 + lane * 4 has a zero byte 1, and one prmt replaces that
+// byte with code byte j of a word: the entry address in one instruction.
 __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lut_lane,
                                                 uint32_t* out) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
@@ -129,7 +155,7 @@ __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lu
         for (int i = 0; i < 4; ++i) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t a = prmt(w[i], 0u, 0x4404u | (j << 4)) + lut_lane;
+                const uint32_t a = prmt(w[i], lut_lane, 0x7604u | (j << 4));
                 out[4 * i + j] = bmul2(lds32(a), sf);
             }
         }
@@ -149,12 +175,18 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     using C = Cfg<NT, TT>;
     const int SC = args.code_stages, SA = args.act_stages;
     const Layout Ly = make_layout(C::kActStage, SC, SA, args.K);
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-    uint8_t* codes = smem + Ly.codes_off;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // the layout assumes dynamic shared memory at window address 1024 (see Layout)
+    if (smem_u32(smem) != kWindowBase) {
+        if (threadIdx.x == 0) record_status(args.status, MXFP4_ERR_CUDA);
+        return;
+    }
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kLutOff);
     uint8_t* acts = smem + Ly.acts_off;
+    auto codes_stage = [&](int i) {
+        return i < Ly.n_codes_lo ? smem + Ly.codes_lo_off + i * kCodeBytes
+                                 : smem + Ly.codes_hi_off + (i - Ly.n_codes_lo) * kCodeBytes;
+    };
     uint8_t* scales = smem + Ly.scales_off;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bar_off);
     uint64_t* cfull = bars;                          // codes stage landed (TMA tx)
@@ -266,7 +298,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 for (int si = 0; si < nss; ++si) {
                     const int ss = si + rot < nss ? si + rot : si + rot - nss;
                     if (!mbar_wait(&cempty[c.idx], c.ph ^ 1, s_abort)) { ok = false; break; }
-                    uint8_t* dst = codes + c.idx * kCodeBytes;
+                    uint8_t* dst = codes_stage(c.idx);
                     mbar_arrive_expect_tx(&cfull[c.idx], kCodeBytes);
                     const int x = ss * kCodeRowBytes;
                     if (MODE == EPI_SWIGLU) {
@@ -441,7 +473,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 if (si == 0) got = got && mbar_wait(&sfull[lt & 1], (lt >> 1) & 1, s_abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t row_addr = smem_u32(codes + c.idx * kCodeBytes) + srow * kCodeRowBytes;
+                const uint32_t row_addr = smem_u32(codes_stage(c.idx)) + srow * kCodeRowBytes;
                 int done = 0;
                 for (int j = 0; j < nsub; ++j, ++kit) {
                     const int xs = C::kLock ? a.idx * kSub + j : xr.idx;
@@ -581,7 +613,7 @@ int64_t max_gemm_k() {
 }
 
 // Host launcher.  `tmap_w` covers the codes as a 3-D tensor {K/2, rows_w, G}
-// with box {32, 64 (SWIGLU) or 128, 1} and 32B swizzle; `tmap_x` covers the
+// with box {128, 64 (SWIGLU) or 128, 1} and 128B swizzle; `tmap_x` covers the
 // activations {K, rows} (bf16) with box {64, nt} and 128B swizzle.
 cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,

@@ -59,6 +59,8 @@ def test_gemm_argument_checks(lib):
     assert g(A, 0, 256, A, A, 512, A, 0, N, 0, N) == _lib.ERR_INVALID_ARG
     assert g(A, 8, 256, A, A, 512, A, 5, N, 0, N) == _lib.ERR_INVALID_ARG
     assert g(A, 8, 96, A, A, 512, A, 0, N, 0, N) == _lib.ERR_UNSUPPORTED_SHAPE
+    # the largest K is 7680 (the tile's block scales are staged whole in shared memory)
+    assert g(A, 8, 7680 + 64, A, A, 512, A, 0, N, 0, N) == _lib.ERR_UNSUPPORTED_SHAPE
     assert g(A, 8, 256, U, A, 512, A, 0, N, 0, N) == _lib.ERR_MISALIGNED
     assert g(A, 8, 256, A, A, 512, A, 1, N, 0, N) == _lib.ERR_WORKSPACE   # W4A4 needs ws
     assert lib.mxfp4_gemm_workspace_size(8, 256, 512, 0) == 0
