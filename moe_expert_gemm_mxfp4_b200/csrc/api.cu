@@ -307,7 +307,8 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     mxfp4_status st = device_info(&d);
     if (st != MXFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const mx::TokenTiling tiling = mx::pick_token_tiling(M, 1);
+    const mx::TokenTiling tiling =
+        mode == MXFP4_W4A4 ? mx::pick_token_tiling_w4a4(M, 1) : mx::pick_token_tiling(M, 1);
     CUtensorMap tw, tx;
     if ((st = encode_codes_map(&tw, w_codes, K, N, 1, 128)) != MXFP4_OK) return st;
     uint8_t* xq_codes = static_cast<uint8_t*>(ws);
@@ -433,7 +434,7 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
     if (e != cudaSuccess) return cuda_fail(e);
 
     trace_mark(1, s);
-    const mx::TokenTiling tiling = mx::pick_token_tiling(P, E);
+    const mx::TokenTiling tiling = a4 ? mx::pick_token_tiling_w4a4(P, E) : mx::pick_token_tiling(P, E);
     const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
     const int64_t tok_tiles = (P + tile_rows - 1) / tile_rows + E;
 

@@ -49,8 +49,7 @@ using namespace gemm;
 
 constexpr int kThreads = 512;
 constexpr int kBK = 64;             // K per pipeline stage
-constexpr int kASlots = 8;          // TMEM A-operand slots (32 columns each)
-constexpr int kACol0 = 256;         // first TMEM column of the A slots
+constexpr int kASlots = 8;          // at most 8 TMEM A-operand slots (32 columns each)
 constexpr int kSub = 4;             // 64-wide K sub-stages per codes super-stage
 constexpr int kCodeRowBytes = kSub * kBK / 2;          // 128 B of codes per weight row
 constexpr int kCodeBytes = kBM * kCodeRowBytes;        // one codes super-stage (16 KB)
@@ -68,15 +67,20 @@ struct Cfg {
     static constexpr int kActTile = NT * kBK * 2;          // one token tile of one K stage
     static constexpr int kActStage = TT * kActTile;
     static constexpr int kAccCols = TT * NT;               // TMEM columns of one accumulator set
-    static constexpr int kAccBufs = 2 * kAccCols <= kACol0 ? 2 : 1;
+    // K stages per MMA group (one barrier wait and one commit each): 4, or 2 when the
+    // accumulators need more TMEM (NT = 192: two 192-column buffers + 4 A slots)
+    static constexpr int kGrp = NT * TT > 128 && TT == 1 ? 2 : kSub;
+    static constexpr int kACol = 512 - 2 * kGrp * 32;       // A slots: two sets of kGrp
+    static constexpr int kAccBufs = 2 * kAccCols <= kACol ? 2 : 1;
     static constexpr int kTileRows = TT * NT;               // token rows of a work tile
     // NT <= 64: the activation ring has one stage per A slot and both are released by
     // the same MMA commit (one commit per K stage instead of two).
     static constexpr bool kLock = NT <= 64;
-    static constexpr int kMaxActStages = kLock ? kASlots : (TT == 1 ? 5 : kSub);
+    static constexpr int kMaxActStages = kLock ? kASlots : (TT == 1 ? (NT > 128 ? 4 : 5) : kSub);
     static constexpr int kChunk = kAccCols < 32 ? kAccCols : 32;   // epilogue columns per TMEM load
     static_assert(kActTile % 1024 == 0, "activation tiles must keep 1024-B alignment");
-    static_assert(kAccCols <= kACol0, "accumulators overlap the A slots");
+    static_assert(kAccCols <= kACol, "accumulators overlap the A slots");
+    static_assert(!kLock || kGrp == kSub, "the locked activation ring follows groups of kSub stages");
 };
 
 // Shared-memory layout, identical on host (sizing) and device.  Offsets count from
@@ -222,7 +226,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
             mbar_init(&xempty[s], 1);
         }
         for (int a = 0; a < kASlots; ++a) {
-            mbar_init(&afull[a], 512);   // per group: 2 arrivals x 256 dequant threads
+            mbar_init(&afull[a], 256 * C::kGrp / 2);   // per group: kGrp/2 arrivals x 256 dequant threads
             mbar_init(&aempty[a], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -406,29 +410,32 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * C::kAccCols;
                 int ki = 0;
-                for (int si = 0; si < nss; ++si) {
+                for (int si = 0; si < nss && ok; ++si) {
                     const int ss = si + rot < nss ? si + rot : si + rot - nss;
                     const int nsub = min(kSub, nk - ss * kSub);
-                    if (!mbar_wait(&afull[a.idx], a.ph, s_abort)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int j = 0; j < nsub; ++j, ++ki) {
-                        const int xs = C::kLock ? a.idx * kSub + j : x.idx;
-                        const uint32_t b_base = smem_u32(acts + xs * C::kActStage);
-                        const uint32_t a_tmem = tmem_base + kACol0 + (a.idx * kSub + j) * 32;
+                    for (int g0 = 0; g0 < nsub; g0 += C::kGrp) {
+                        const int ng = min(C::kGrp, nsub - g0);
+                        if (!mbar_wait(&afull[a.idx], a.ph, s_abort)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int j = 0; j < ng; ++j, ++ki) {
+                            const int xs = C::kLock ? a.idx * kSub + j : x.idx;
+                            const uint32_t b_base = smem_u32(acts + xs * C::kActStage);
+                            const uint32_t a_tmem = tmem_base + C::kACol + (a.idx * C::kGrp + j) * 32;
 #pragma unroll
-                        for (int tt = 0; tt < TT; ++tt)
+                            for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-                            for (int jj = 0; jj < 4; ++jj)
-                                mma_bf16_ts(d_tmem + tt * NT, a_tmem + 8 * jj,
-                                            sw128_desc(b_base + tt * C::kActTile + 32 * jj), idesc,
-                                            (ki | jj) != 0 ? 1u : 0u);
-                        if (!C::kLock) {
-                            tc_commit(&xempty[x.idx]);
-                            x.next(SA);
+                                for (int jj = 0; jj < 4; ++jj)
+                                    mma_bf16_ts(d_tmem + tt * NT, a_tmem + 8 * jj,
+                                                sw128_desc(b_base + tt * C::kActTile + 32 * jj), idesc,
+                                                (ki | jj) != 0 ? 1u : 0u);
+                            if (!C::kLock) {
+                                tc_commit(&xempty[x.idx]);
+                                x.next(SA);
+                            }
                         }
+                        tc_commit(&aempty[a.idx]);
+                        a.next(2);
                     }
-                    tc_commit(&aempty[a.idx]);
-                    a.next(2);
                 }
                 if (!ok) break;
                 tc_commit(&accfull[b]);
@@ -456,7 +463,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
             srow = q * 32 + lane;
         }
         const uint32_t sw = static_cast<uint32_t>(srow) & 7u;   // 128B swizzle: chunk ^= row % 8
-        const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
+        const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::kACol;
         RingPos c, a, xr;        // codes super-stages, A-slot sets, activation stages (!kLock)
         int kit = 0, lt = 0;
         bool ok = true;
@@ -467,43 +474,55 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
             for (int si = 0; si < nss && ok; ++si) {
                 const int ss = si + rot < nss ? si + rot : si + rot - nss;
                 const int nsub = min(kSub, nk - ss * kSub);
-                // the group's A slots are free, its codes have landed, the tile's scales too
-                bool got = mbar_wait(&aempty[a.idx], a.ph ^ 1, s_abort) &&
-                           mbar_wait(&cfull[c.idx], c.ph, s_abort);
+                // the super-stage's codes have landed, the tile's scales too
+                bool got = mbar_wait(&cfull[c.idx], c.ph, s_abort);
                 if (si == 0) got = got && mbar_wait(&sfull[lt & 1], (lt >> 1) & 1, s_abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
-                tc_fence_after();
                 const uint32_t row_addr = smem_u32(codes_stage(c.idx)) + srow * kCodeRowBytes;
-                int done = 0;
-                for (int j = 0; j < nsub; ++j, ++kit) {
-                    const int xs = C::kLock ? a.idx * kSub + j : xr.idx;
-                    const uint32_t xph = C::kLock ? a.ph : xr.ph;
-                    if ((kit & 1) == d) {
-                        const int ks = ss * kSub + j;
-                        const uint32_t sc = valid ? lds_u16(sc_row + 2 * ks) : 0x7F7Fu;
-                        const uint4 c0 = lds128(row_addr + (((2u * j) ^ sw) << 4));
-                        const uint4 c1 = lds128(row_addr + (((2u * j + 1u) ^ sw) << 4));
-                        uint32_t out[32];
-                        dequant_block16(c0, sc & 0xFFu, lut_lane, out);
-                        dequant_block16(c1, sc >> 8, lut_lane, out + 16);
-                        tmem_st_x32(tmem_lane + (a.idx * kSub + j) * 32, out);
-                        tmem_wait_st();
-                        // the stage's activation tile must have landed too: the MMA issuer
-                        // waits on the group barrier only
-                        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&xfull[xs], xph, s_abort))) { ok = false; break; }
-                        tc_fence_before();
-                        mbar_arrive(&afull[a.idx]);
-                        ++done;
+                for (int g0 = 0; g0 < nsub; g0 += C::kGrp) {
+                    const int ng = min(C::kGrp, nsub - g0);
+                    // the group's A slots are free
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&aempty[a.idx], a.ph ^ 1, s_abort))) { ok = false; break; }
+                    tc_fence_after();
+                    int done = 0;
+                    int xs0 = 0, xs1 = 0;
+                    uint32_t xph0 = 0, xph1 = 0;
+                    for (int jg = 0; jg < ng; ++jg, ++kit) {
+                        const int j = g0 + jg;    // stage within the super-stage
+                        if ((kit & 1) == d) {
+                            const int ks = ss * kSub + j;
+                            const uint32_t sc = valid ? lds_u16(sc_row + 2 * ks) : 0x7F7Fu;
+                            const uint4 c0 = lds128(row_addr + (((2u * j) ^ sw) << 4));
+                            const uint4 c1 = lds128(row_addr + (((2u * j + 1u) ^ sw) << 4));
+                            uint32_t out[32];
+                            dequant_block16(c0, sc & 0xFFu, lut_lane, out);
+                            dequant_block16(c1, sc >> 8, lut_lane, out + 16);
+                            tmem_st_x32(tmem_lane + (a.idx * C::kGrp + jg) * 32, out);
+                            const int xs = C::kLock ? a.idx * kSub + jg : xr.idx;
+                            const uint32_t xph = C::kLock ? a.ph : xr.ph;
+                            if (done == 0) { xs0 = xs; xph0 = xph; } else { xs1 = xs; xph1 = xph; }
+                            ++done;
+                        }
+                        if (!C::kLock) xr.next(SA);
                     }
-                    if (!C::kLock) xr.next(SA);
+                    // The MMA issuer waits for the whole group, so this thread signals its
+                    // stages together at the end: one wait for all of its TMEM stores, and
+                    // the activation tiles of its stages must have landed too.
+                    tmem_wait_st();
+                    bool landed = true;
+                    if (done > 0) landed = mbar_wait(&xfull[xs0], xph0, s_abort);
+                    if (done > 1) landed = landed && mbar_wait(&xfull[xs1], xph1, s_abort);
+                    if (!__all_sync(0xFFFFFFFFu, landed)) { ok = false; break; }
+                    tc_fence_before();
+                    // every dequant thread arrives kGrp/2 times per group (the warpgroups
+                    // alternate stages; short groups count the same)
+#pragma unroll
+                    for (int i2 = 0; i2 < C::kGrp / 2; ++i2) mbar_arrive(&afull[a.idx]);
+                    a.next(2);
                 }
                 if (!ok) break;
-                // every dequant thread arrives exactly twice per group (a group has four
-                // stages, two per warpgroup); short groups are topped up here
-                for (; done < 2; ++done) mbar_arrive(&afull[a.idx]);
-                mbar_arrive(&cempty[c.idx]);     // this warpgroup is done with the super-stage
+                mbar_arrive(&cempty[c.idx]);     // this warpgroup is done reading the codes
                 c.next(SC);
-                a.next(2);
             }
         }
         if (!ok) {
@@ -546,12 +565,12 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
 template <int NT, int TT>
 bool ring_depths(int K, int* sc, int* sa, int* smem) {
     using C = Cfg<NT, TT>;
-    // The activation ring must hold at least one whole group of kSub stages: the MMA
+    // The activation ring must hold at least one whole group of kGrp stages: the MMA
     // issuer consumes a group only once all its stages are ready.
     int c = C::kLock ? kMaxCodeStagesLock : kMaxCodeStages, a = C::kMaxActStages;
     while (make_layout(C::kActStage, c, a, K).total > kSmemLimit) {
         if (c > 2) --c;
-        else if (!C::kLock && a > kSub) --a;
+        else if (!C::kLock && a > C::kGrp) --a;
         else return false;
     }
     *sc = c;
@@ -580,6 +599,10 @@ cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap
     if (nt == 16) return launch_cfg<16, 1, MODE>(tw, tx, a, grid, stream);
     if (nt == 32) return launch_cfg<32, 1, MODE>(tw, tx, a, grid, stream);
     if (nt == 64) return launch_cfg<64, 1, MODE>(tw, tx, a, grid, stream);
+    if (nt == 192) {
+        int sc, sa, smem;
+        if (ring_depths<192, 1>(a.K, &sc, &sa, &smem)) return launch_cfg<192, 1, MODE>(tw, tx, a, grid, stream);
+    }
     if (tt == 2) {   // two token tiles per weight tile when their rings fit this K
         int sc, sa, smem;
         if (ring_depths<128, 2>(a.K, &sc, &sa, &smem)) return launch_cfg<128, 2, MODE>(tw, tx, a, grid, stream);
@@ -596,6 +619,10 @@ TokenTiling pick_token_tiling(int64_t rows, int64_t groups) {
     if (avg <= 16) return {16, 1};
     if (avg <= 32) return {32, 1};
     if (avg <= 64) return {64, 1};
+    // 192-row token tiles dequantize each weight tile once per 192 tokens instead of
+    // 128 (the dequantize work bounds the large-batch GEMM), at the cost of a ragged
+    // last tile per expert: worth it once experts average a few tiles
+    if (avg >= 320) return {192, 1};
     return {128, 1};
 }
 

@@ -15,16 +15,16 @@
 // Work tile: 128 weight rows (the MMA's M) x NT token rows (N); K in super-stages
 // of 256 (128 bytes of codes per row, one 128B-swizzle row), four MMAs of K = 64.
 //
-// Roles (one persistent CTA per SM, 8 warps):
+// Roles (one persistent CTA per SM, 12 warps; warp 3 idles):
 //   warp 0    weight producer: per tile the block scales of its 128 rows (bulk
 //             copy, double-buffered); per super-stage the codes box -> stage ring.
 //   warp 2    activation producer: per tile the block scales of its NT rows (bulk
 //             copy of the covering 16-byte-aligned range, double-buffered); per
 //             super-stage the activation codes box -> stage ring.
-//   warp 3    scale builder: per super-stage rewrites both operands' scales into
-//             the tensor core's scale-factor layout (per 4 scales of a 128-row
-//             block: row r at byte 16 (r % 32) + 4 (r / 32) + j), waits for the
-//             stage's codes and marks the stage ready.
+//   warps 8-11 scale builders: per super-stage each rewrites one operand's four
+//             scales per row into the tensor core's scale-factor layout (per 4
+//             scales of a 128-row block: row r at byte 16 (r % 32) + 4 (r / 32) + j),
+//             waits for that operand's codes and marks its part of the stage ready.
 //   warp 1    MMA issuer: per super-stage copies the four scale atoms to TMEM
 //             (tcgen05.cp, ordered with its MMAs), issues the MMAs, and releases
 //             the stage with one commit.
@@ -39,7 +39,7 @@ namespace {
 
 using namespace gemm;
 
-constexpr int kThreads4 = 256;
+constexpr int kThreads4 = 384;
 constexpr int kSSK = 256;                    // K per super-stage
 constexpr int kRowBytes = kSSK / 2;          // codes bytes per row per super-stage
 constexpr int kWBytes = kBM * kRowBytes;     // weight codes per stage (16 KB)
@@ -146,14 +146,14 @@ grouped_w4a4_kernel(const __grid_constant__ CUtensorMap tmap_w,
         for (int s = 0; s < S; ++s) {
             mbar_init(&wfull[s], 1);
             mbar_init(&xfull[s], 1);
-            mbar_init(&ready[s], 1);
+            mbar_init(&ready[s], 4);   // one arrival per scale-builder warp
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sfull[b], 1);
-            mbar_init(&sempty[b], 1);
+            mbar_init(&sempty[b], 2);    // the two weight-scale builders
             mbar_init(&xsfull[b], 1);
-            mbar_init(&xsempty[b], 1);
+            mbar_init(&xsempty[b], 2);   // the two token-scale builders
             mbar_init(&accfull[b], 1);
             mbar_init(&accempty[b], 128);
         }
@@ -282,8 +282,12 @@ grouped_w4a4_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 ps.drain(xsfull, 2, s_never);
             }
         }
-    } else if (warp == 3) {
-        // ---------------- scale builder
+    } else if (warp >= 8) {
+        // ---------------- scale builders: warp 8 + (operand * 2 + h) writes the atom of
+        // scales 4h .. 4h+3 of the super-stage for operand 0 (weights, A) or 1 (tokens, B)
+        const int bw = warp - 8;
+        const bool is_b = bw >= 2;
+        const int h = bw & 1;
         RingPos c;
         int lt = 0;
         bool ok = true;
@@ -291,49 +295,44 @@ grouped_w4a4_kernel(const __grid_constant__ CUtensorMap tmap_w,
             const TileInfo ti = decode_tile(t, s_tstart, s_off, G, NT);
             const int sb = lt & 1;
             const uint32_t tph = (lt >> 1) & 1;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[sb], tph, s_abort) &&
-                                             mbar_wait(&xsfull[sb], tph, s_abort))) { ok = false; break; }
-            const uint32_t wrow0 = smem_u32(wsc + sb * Ly.wsc_bytes);
-            const uint32_t xrow0 = smem_u32(xsc + sb * Ly.xsc_bytes) + s_xshift[sb];
-            // this lane's rows: r = lane + 32 m1 (m1 = 0..3), for A (weights) and B (tokens)
-            uint32_t arow[4], brow[4];
-            bool avalid[4], bvalid[4];
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(is_b ? &xsfull[sb] : &sfull[sb], tph, s_abort))) {
+                ok = false;
+                break;
+            }
+            // this lane's rows r = lane + 32 m1 (m1 = 0..3) of the operand
+            uint32_t row[4];
+            bool valid[4];
+            const uint32_t base = is_b ? smem_u32(xsc + sb * Ly.xsc_bytes) + s_xshift[sb]
+                                       : smem_u32(wsc + sb * Ly.wsc_bytes);
 #pragma unroll
             for (int m1 = 0; m1 < 4; ++m1) {
                 const int r = lane + 32 * m1;
-                const int srow = MODE == EPI_SWIGLU ? swiglu_staged_row(r) : r;
-                avalid[m1] = MODE == EPI_SWIGLU || ti.f * kBM + r < args.rows_w;
-                arow[m1] = wrow0 + srow * kb;
-                bvalid[m1] = r < ti.mrows;
-                brow[m1] = xrow0 + r * kb;
+                if (is_b) {
+                    valid[m1] = r < ti.mrows;
+                    row[m1] = base + r * kb;
+                } else {
+                    valid[m1] = MODE == EPI_SWIGLU || ti.f * kBM + r < args.rows_w;
+                    row[m1] = base + (MODE == EPI_SWIGLU ? swiglu_staged_row(r) : r) * kb;
+                }
             }
             for (int si = 0; si < nss; ++si) {
                 const int ss = ss_of(si);
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[c.idx], c.ph ^ 1, s_abort))) { ok = false; break; }
-                const uint32_t atoms = smem_u32(smem + c.idx * Ly.stage_bytes + Ly.atoms_off);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int k0 = 8 * ss + 4 * h;
-                    sts128(atoms + h * kAtom + 16 * lane, scale_word(arow[0], k0, kb, avalid[0]),
-                           scale_word(arow[1], k0, kb, avalid[1]), scale_word(arow[2], k0, kb, avalid[2]),
-                           scale_word(arow[3], k0, kb, avalid[3]));
-                    sts128(atoms + (2 + h) * kAtom + 16 * lane, scale_word(brow[0], k0, kb, bvalid[0]),
-                           scale_word(brow[1], k0, kb, bvalid[1]), scale_word(brow[2], k0, kb, bvalid[2]),
-                           scale_word(brow[3], k0, kb, bvalid[3]));
-                }
+                const uint32_t atom = smem_u32(smem + c.idx * Ly.stage_bytes + Ly.atoms_off) + bw * kAtom;
+                const int k0 = 8 * ss + 4 * h;
+                sts128(atom + 16 * lane, scale_word(row[0], k0, kb, valid[0]),
+                       scale_word(row[1], k0, kb, valid[1]), scale_word(row[2], k0, kb, valid[2]),
+                       scale_word(row[3], k0, kb, valid[3]));
                 // generic-proxy writes -> visible to the tensor core's (async-proxy) tcgen05.cp
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                const bool got = mbar_wait(&wfull[c.idx], c.ph, s_abort) && mbar_wait(&xfull[c.idx], c.ph, s_abort);
+                const bool got = mbar_wait(is_b ? &xfull[c.idx] : &wfull[c.idx], c.ph, s_abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 if (lane == 0) mbar_arrive(&ready[c.idx]);
                 c.next(S);
             }
             if (!ok) break;
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sempty[sb]);
-                mbar_arrive(&xsempty[sb]);
-            }
+            if (lane == 0) mbar_arrive(is_b ? &xsempty[sb] : &sempty[sb]);
         }
         if (!ok) {
             *s_abort = 1;
@@ -386,7 +385,7 @@ grouped_w4a4_kernel(const __grid_constant__ CUtensorMap tmap_w,
             tc_commit(drain);
             mbar_wait(drain, 0, s_never);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4) {   // warps 4-7
         // ---------------- epilogue warpgroup
         const int q = warp & 3;
         int lt = 0;
@@ -445,13 +444,25 @@ cudaError_t launch4(const CUtensorMap& tw, const CUtensorMap& tx, GemmArgs a, in
 template <int MODE>
 cudaError_t launch4_mode(int nt, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                          int grid, cudaStream_t stream) {
+    // nt must match the activation map's box rows (the stage expects nt * 128 bytes)
     if (nt == 16) return launch4<16, MODE>(tw, tx, a, grid, stream);
     if (nt == 32) return launch4<32, MODE>(tw, tx, a, grid, stream);
     if (nt == 64) return launch4<64, MODE>(tw, tx, a, grid, stream);
-    return launch4<128, MODE>(tw, tx, a, grid, stream);
+    if (nt == 128) return launch4<128, MODE>(tw, tx, a, grid, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
+
+// Token tiling of the W4A4 engine: NT rows per MMA (16..128) from the mean rows
+// per group.
+TokenTiling pick_token_tiling_w4a4(int64_t rows, int64_t groups) {
+    const int64_t avg = (rows + groups - 1) / (groups > 0 ? groups : 1);
+    if (avg <= 16) return {16, 1};
+    if (avg <= 32) return {32, 1};
+    if (avg <= 64) return {64, 1};
+    return {128, 1};
+}
 
 int64_t max_gemm_k_w4a4() {
     int64_t k = 256;

@@ -57,6 +57,7 @@ cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap&
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream);
 int64_t max_gemm_k_w4a4();   // largest contraction length the W4A4 engine accepts
+TokenTiling pick_token_tiling_w4a4(int64_t rows, int64_t groups);
 cudaError_t launch_grouped_gemm_w4a4(int mode, int nt, const CUtensorMap& tmap_w,
                                      const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                      cudaStream_t stream);

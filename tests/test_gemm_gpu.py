@@ -31,7 +31,8 @@ def test_gemm_small_workload():
 
 @pytest.mark.parametrize("M,K,N", [(1, 64, 1), (3, 64, 130), (16, 128, 128), (17, 192, 200),
                                    (40, 256, 256), (64, 320, 384), (100, 512, 129),
-                                   (257, 704, 640), (1024, 2880, 2880)])
+                                   (257, 704, 640), (500, 512, 384), (777, 1024, 256),
+                                   (1024, 2880, 2880)])
 def test_gemm_shapes(M, K, N):
     g = torch.Generator().manual_seed(M * 7 + K + N)
     x = torch.randn(M, K, generator=g).to(torch.bfloat16)
