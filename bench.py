@@ -441,6 +441,37 @@ def traffic_record(kernel, workload):
     return r.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------------ profiling driver
+
+def run_profile_case(args):
+    """The calls of one breakdown workload, for an ncu capture of its kernels."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    mx._lib.load()
+    dev = torch.device("cuda", 0)
+    n = args.warmup + args.steps
+    if args.profile == "quant":
+        x = inputs.quant_tensor().to(dev)
+        for _ in range(n):
+            c, sc = mx.mxfp4_quantize(x)
+            mx.mxfp4_dequantize(c, sc)
+    else:
+        cfg = inputs.MOE_CONFIGS["moe_decode" if args.profile == "decode" else "moe_120b"]
+        mode = mx.W4A16 if args.profile == "decode" else mx.W4A4
+        L = gpu_layer(cfg, dev)
+        xd, ld = L["x"].to(dev), L["logits"].to(dev)
+        out = torch.empty((xd.shape[0], cfg.H), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((mx.moe_mxfp4_workspace_size(xd.shape[0], cfg.H, cfg.I, cfg.E, cfg.top_k, mode),),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(n):
+            mx.moe_mxfp4_mlp(xd, ld, cfg.top_k, *L["w"], mode=mode, out=out, ws=ws)
+    torch.cuda.synchronize()
+    status = mx.mxfp4_get_device_status()
+    print(json.dumps({"profile": args.profile, "calls": n, "device_status": status}), flush=True)
+    if status != 0:
+        sys.exit(1)
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -453,12 +484,18 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the prefill workload (profiling runs on a smaller case)")
+    ap.add_argument("--profile", choices=["decode", "w4a4_120b", "quant"], default=None,
+                    help="run one breakdown workload --warmup + --steps times, untimed, and "
+                         "print a status line (a driver for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.profile:
+        run_profile_case(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

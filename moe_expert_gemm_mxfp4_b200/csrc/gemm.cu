@@ -73,14 +73,17 @@ struct Cfg {
     static constexpr int kACol = 512 - 2 * kGrp * 32;       // A slots: two sets of kGrp
     static constexpr int kAccBufs = 2 * kAccCols <= kACol ? 2 : 1;
     static constexpr int kTileRows = TT * NT;               // token rows of a work tile
-    // NT <= 64: the activation ring has one stage per A slot and both are released by
-    // the same MMA commit (one commit per K stage instead of two).
+    // NT <= 64 (decode): the activation ring holds whole groups (chunks of kSub
+    // stages), each filled by one barrier and released by one MMA commit per group,
+    // several groups ahead of the MMA (an activation tile's load latency exceeds a
+    // group's MMA time at this N).  Otherwise the ring holds single stages.
     static constexpr bool kLock = NT <= 64;
-    static constexpr int kMaxActStages = kLock ? kASlots : (TT == 1 ? (NT > 128 ? 4 : 5) : kSub);
+    static constexpr int kActUnit = kLock ? kSub * kActStage : kActStage;   // bytes per ring slot
+    static constexpr int kMaxActStages = kLock ? 4 : (TT == 1 ? (NT > 128 ? 4 : 5) : kSub);
     static constexpr int kChunk = kAccCols < 32 ? kAccCols : 32;   // epilogue columns per TMEM load
     static_assert(kActTile % 1024 == 0, "activation tiles must keep 1024-B alignment");
     static_assert(kAccCols <= kACol, "accumulators overlap the A slots");
-    static_assert(!kLock || kGrp == kSub, "the locked activation ring follows groups of kSub stages");
+    static_assert(!kLock || kGrp == kSub, "the chunked activation ring follows groups of kSub stages");
 };
 
 // Shared-memory layout, identical on host (sizing) and device.  Offsets count from
@@ -178,7 +181,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
     using C = Cfg<NT, TT>;
     const int SC = args.code_stages, SA = args.act_stages;
-    const Layout Ly = make_layout(C::kActStage, SC, SA, args.K);
+    const Layout Ly = make_layout(C::kActUnit, SC, SA, args.K);
     extern __shared__ __align__(1024) uint8_t smem[];
     // the layout assumes dynamic shared memory at window address 1024 (see Layout)
     if (smem_u32(smem) != kWindowBase) {
@@ -332,7 +335,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
     } else if (warp == 2) {
         // ---------------- activation producer
         if (lane == 0) {
-            RingPos x;             // kLock: ring of A-slot sets (2); else: ring of stages (SA)
+            RingPos x;             // kLock: ring of SA group chunks; else: ring of SA stages
             int issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
@@ -341,21 +344,15 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                     const int ss = si + rot < nss ? si + rot : si + rot - nss;
                     const int nsub = min(kSub, nk - ss * kSub);
                     if (C::kLock) {
-                        // one slot per stage of the group, released with the group's A slots
-                        if (!mbar_wait(&aempty[x.idx], x.ph ^ 1, s_abort)) { ok = false; break; }
-                        for (int j = 0; j < kSub; ++j) {
-                            const int slot = x.idx * kSub + j;
-                            if (j < nsub) {
-                                mbar_arrive_expect_tx(&xfull[slot], C::kActStage);
+                        // the group's stages in one chunk: one barrier, one release
+                        if (!mbar_wait(&xempty[x.idx], x.ph ^ 1, s_abort)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&xfull[x.idx], nsub * C::kActStage);
+                        for (int j = 0; j < nsub; ++j)
 #pragma unroll
-                                for (int tt = 0; tt < TT; ++tt)
-                                    tma_load_2d(acts + slot * C::kActStage + tt * C::kActTile, &tmap_x, &xfull[slot],
-                                                (ss * kSub + j) * kBK, ti.row0 + tt * NT);
-                            } else {
-                                mbar_arrive(&xfull[slot]);   // unused slot of a short group: keep phases aligned
-                            }
-                        }
-                        x.next(2);
+                            for (int tt = 0; tt < TT; ++tt)
+                                tma_load_2d(acts + x.idx * C::kActUnit + j * C::kActStage + tt * C::kActTile,
+                                            &tmap_x, &xfull[x.idx], (ss * kSub + j) * kBK, ti.row0 + tt * NT);
+                        x.next(SA);
                         ++issued;
                     } else {
                         for (int j = 0; j < nsub; ++j) {
@@ -375,21 +372,11 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 *s_abort = 1;
                 record_status(args.status, MXFP4_ERR_TIMEOUT);
                 // let the copies already issued land before the CTA exits
-                if (C::kLock) {
-                    RingPos r;
-                    const int first = issued > 2 ? issued - 2 : 0;
-                    for (int i = 0; i < issued; ++i) {
-                        if (i >= first)
-                            for (int j = 0; j < kSub; ++j) mbar_wait(&xfull[r.idx * kSub + j], r.ph, s_never);
-                        r.next(2);
-                    }
-                } else {
-                    RingPos r;
-                    const int first = issued > SA ? issued - SA : 0;
-                    for (int i = 0; i < issued; ++i) {
-                        if (i >= first) mbar_wait(&xfull[r.idx], r.ph, s_never);
-                        r.next(SA);
-                    }
+                RingPos r;
+                const int first = issued > SA ? issued - SA : 0;
+                for (int i = 0; i < issued; ++i) {
+                    if (i >= first) mbar_wait(&xfull[r.idx], r.ph, s_never);
+                    r.next(SA);
                 }
             }
         }
@@ -400,7 +387,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         // of the MMAs in flight, so it is paid once per group, not once per stage.
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kBM, NT);
-            RingPos x, a;          // x: activation stages (only when !kLock); a: A-slot sets
+            RingPos x, a;          // x: activation ring (chunks when kLock, else stages); a: A-slot sets
             int lt = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
@@ -418,8 +405,8 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         if (!mbar_wait(&afull[a.idx], a.ph, s_abort)) { ok = false; break; }
                         tc_fence_after();
                         for (int j = 0; j < ng; ++j, ++ki) {
-                            const int xs = C::kLock ? a.idx * kSub + j : x.idx;
-                            const uint32_t b_base = smem_u32(acts + xs * C::kActStage);
+                            const uint32_t b_base = smem_u32(acts + x.idx * C::kActUnit +
+                                                             (C::kLock ? j * C::kActStage : 0));
                             const uint32_t a_tmem = tmem_base + C::kACol + (a.idx * C::kGrp + j) * 32;
 #pragma unroll
                             for (int tt = 0; tt < TT; ++tt)
@@ -435,6 +422,10 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         }
                         tc_commit(&aempty[a.idx]);
                         a.next(2);
+                        if (C::kLock) {
+                            tc_commit(&xempty[x.idx]);
+                            x.next(SA);
+                        }
                     }
                 }
                 if (!ok) break;
@@ -464,7 +455,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
         }
         const uint32_t sw = static_cast<uint32_t>(srow) & 7u;   // 128B swizzle: chunk ^= row % 8
         const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::kACol;
-        RingPos c, a, xr;        // codes super-stages, A-slot sets, activation stages (!kLock)
+        RingPos c, a, xr;        // codes super-stages, A-slot sets, activation ring
         int kit = 0, lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
@@ -498,8 +489,8 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                             dequant_block16(c0, sc & 0xFFu, lut_lane, out);
                             dequant_block16(c1, sc >> 8, lut_lane, out + 16);
                             tmem_st_x32(tmem_lane + (a.idx * C::kGrp + jg) * 32, out);
-                            const int xs = C::kLock ? a.idx * kSub + jg : xr.idx;
-                            const uint32_t xph = C::kLock ? a.ph : xr.ph;
+                            const int xs = xr.idx;      // kLock: the group's chunk
+                            const uint32_t xph = xr.ph;
                             if (done == 0) { xs0 = xs; xph0 = xph; } else { xs1 = xs; xph1 = xph; }
                             ++done;
                         }
@@ -519,6 +510,7 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
 #pragma unroll
                     for (int i2 = 0; i2 < C::kGrp / 2; ++i2) mbar_arrive(&afull[a.idx]);
                     a.next(2);
+                    if (C::kLock) xr.next(SA);
                 }
                 if (!ok) break;
                 mbar_arrive(&cempty[c.idx]);     // this warpgroup is done reading the codes
@@ -568,14 +560,15 @@ bool ring_depths(int K, int* sc, int* sa, int* smem) {
     // The activation ring must hold at least one whole group of kGrp stages: the MMA
     // issuer consumes a group only once all its stages are ready.
     int c = C::kLock ? kMaxCodeStagesLock : kMaxCodeStages, a = C::kMaxActStages;
-    while (make_layout(C::kActStage, c, a, K).total > kSmemLimit) {
+    const int amin = C::kLock ? 2 : C::kGrp;   // two chunks, or one group of stages
+    while (make_layout(C::kActUnit, c, a, K).total > kSmemLimit) {
         if (c > 2) --c;
-        else if (!C::kLock && a > C::kGrp) --a;
+        else if (a > amin) --a;
         else return false;
     }
     *sc = c;
     *sa = a;
-    *smem = make_layout(C::kActStage, c, a, K).total;
+    *smem = make_layout(C::kActUnit, c, a, K).total;
     return true;
 }
 

@@ -209,10 +209,22 @@ route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
             inv[p] = static_cast<int32_t>(pos);
             if (w_sorted) w_sorted[pos] = weights[p];
         }
-        if (x) {
+        if (x) {   // all of a lane's loads first, then its stores: 8 x 16 B in flight per lane
             const uint4* src = x + t * row_vec;
             uint4* dst = x_sorted + pos * row_vec;
-            for (int64_t c = lane; c < row_vec; c += 32) dst[c] = __ldg(src + c);
+            for (int64_t c0 = 0; c0 < row_vec; c0 += 32 * 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int64_t c = c0 + lane + 32 * u;
+                    if (c < row_vec) v[u] = __ldg(src + c);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int64_t c = c0 + lane + 32 * u;
+                    if (c < row_vec) dst[c] = v[u];
+                }
+            }
         }
         if (xs) {
             const uint8_t* src = xs + t * xs_row;
