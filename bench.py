@@ -525,7 +525,7 @@ def main():
     st = r["stage_ms"]
     gu_flops = 2.0 * cfg.T * cfg.top_k * 2 * cfg.I * cfg.H
     achieved = gu_flops / st["gate_up"] / 1e9
-    roof = {"kernel": "grouped_w4a16_kernel<128, SWIGLU> (gate/up projection + SwiGLU)",
+    roof = {"kernel": "grouped_w4a16_kernel, gate/up projection + SwiGLU (192-row token tiles at this size)",
             "bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
             "frac": achieved / pk["bf16"],
             "peak_source": f"{pk['source']} bf16 dense (burst; timed region < 1 s)",
