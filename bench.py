@@ -129,12 +129,20 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Max of v over all ranks (NCCL with a device tensor; gloo on the CPU)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(world: int, steps: int, flops_per_step: float, total_ms_max: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank runs `steps` steps of its own
+    layer (replicas, weak scaling), timed by the slowest rank."""
+    return world * steps * flops_per_step / total_ms_max / 1e9
 
 
 # ------------------------------------------------------------------ workload set-up
@@ -521,7 +529,7 @@ def main():
     fl = layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I)
     step_ms = statistics.mean(r["step_ms"])
     total_ms = max_over_ranks(sum(r["step_ms"]), world)
-    value = world * args.steps * fl / total_ms / 1e9
+    value = job_value(world, args.steps, fl, total_ms)
     st = r["stage_ms"]
     gu_flops = 2.0 * cfg.T * cfg.top_k * 2 * cfg.I * cfg.H
     achieved = gu_flops / st["gate_up"] / 1e9

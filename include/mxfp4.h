@@ -189,6 +189,14 @@ MXFP4_API mxfp4_status mxfp4_get_device_status(void* stream);
 MXFP4_API int mxfp4_last_cuda_error(void);
 /* Static, human-readable name of a status code. */
 MXFP4_API const char* mxfp4_status_string(mxfp4_status s);
+/* Failure-detection self-test (no counterpart in the pages): launches one CTA on
+ * `stream` whose only thread waits on an mbarrier that nothing arrives on.  After
+ * the library's wait limit (2 s of %globaltimer) the wait gives up, the kernel
+ * records MXFP4_ERR_TIMEOUT in the device status word and returns, exactly as the
+ * library's kernels do when a pipeline stalls.  No fault, trap or hang: the context
+ * stays usable.  Returns MXFP4_OK once launched (read the outcome with
+ * mxfp4_get_device_status), or MXFP4_ERR_ARCH / MXFP4_ERR_CUDA. */
+MXFP4_API mxfp4_status mxfp4_selftest_wait_timeout(void* stream);
 
 #ifdef __cplusplus
 }

@@ -25,7 +25,7 @@ __all__ = [
     "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_gemm_workspace_size",
     "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
     "moe_mxfp4_workspace_size", "moe_mxfp4_mlp_noalloc", "mxfp4_get_device_status",
-    "mxfp4_set_trace_events",
+    "mxfp4_selftest_wait_timeout", "mxfp4_set_trace_events",
     "Mxfp4Error", "Mxfp4LibraryMissing",
     "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
 ]
@@ -171,6 +171,13 @@ def moe_mxfp4_mlp_noalloc(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13
 def mxfp4_get_device_status(stream=None) -> int:
     """Synchronize the stream and return (and clear) the device status word."""
     return int(_lib.load().mxfp4_get_device_status(_stream(stream)))
+
+
+def mxfp4_selftest_wait_timeout(stream=None):
+    """Launch the failure-detection self-test: one wait that nothing satisfies, which
+    gives up after the library's wait limit and records MXFP4_ERR_TIMEOUT."""
+    _lib.check("mxfp4_selftest_wait_timeout",
+               _lib.load().mxfp4_selftest_wait_timeout(_stream(stream)))
 
 
 _trace_keepalive = None

@@ -59,6 +59,7 @@ _SIGS = {
     "moe_mxfp4_mlp_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
                                              ctypes.c_int, _vp]),
     "mxfp4_get_device_status": (ctypes.c_int, [_vp]),
+    "mxfp4_selftest_wait_timeout": (ctypes.c_int, [_vp]),
     "mxfp4_set_trace_events": (None, [_vp, ctypes.c_int]),
     "mxfp4_last_cuda_error": (ctypes.c_int, []),
     "mxfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),

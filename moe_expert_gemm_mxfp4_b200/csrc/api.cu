@@ -226,6 +226,14 @@ const char* mxfp4_status_string(mxfp4_status s) {
 
 int mxfp4_last_cuda_error(void) { return tl_last_cuda_error; }
 
+mxfp4_status mxfp4_selftest_wait_timeout(void* stream) {
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaError_t e = mx::launch_selftest_wait_timeout(d->status, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
 void mxfp4_set_trace_events(void* const* events, int n_events) {
     tl_trace_events = n_events > 0 ? events : nullptr;
     tl_trace_n = n_events > 0 ? n_events : 0;
