@@ -8,7 +8,7 @@
  * The MoE expert MLP on MXFP4 expert weights is the layer that page runs through
  * its downloadable MoE kernel (section "Zero-Build Kernels from the Hub").
  *
- * Encoding used throughout (the pages leave these open):
+ * Encoding used throughout (readings: the pages leave these open):
  *   - E2M1 with exponent bias 1: magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6};
  *     a 4-bit code is (sign << 3) | magnitude index;
  *   - one E8M0 scale byte S per block, value 2^(S-127), S = 0xFF is NaN;

@@ -20,8 +20,8 @@ The pages fix the E2M1 bit split (1 sign, 2 exponent, 1 mantissa) and that 32
 consecutive elements share one scale ([P4] "What MXFP4 Is"), and that the MoE
 expert MLP runs on MXFP4 weights ([P4] "Zero-Build Kernels from the Hub",
 MegaBlocks MoE).  Everything else (scale encoding, rounding, nibble order,
-routing rule, gated-SiLU expert MLP) is a reading stated at each function and
-listed in DESIGN.md.
+routing rule, gated-SiLU expert MLP) is a reading, stated at the function that
+takes it.
 
 Parity pins: every function here is pinned by ``tests/test_oracle.py`` against
 values the pages fix, closed forms, invariants or brute force.  The one part

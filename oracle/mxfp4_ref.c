@@ -12,7 +12,7 @@
  * section on the zh-CN page and the E2M1 sentence of the otomatix.tech page):
  *   - each element is an E2M1 float: 1 sign bit, 2 exponent bits, 1 mantissa bit;
  *   - elements come in blocks of 32 that share one scale.
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - E2M1 exponent bias 1, so the magnitudes are {0, .5, 1, 1.5, 2, 3, 4, 6};
  *   - the shared scale is an E8M0 byte S meaning 2^(S-127); S = 0xFF is NaN;
  *   - scale exponent s = floor(log2(amax)) - 2 ("floor" rule, 2 being the
