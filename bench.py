@@ -253,11 +253,16 @@ def time_e2e(L, cfg, mode, steps, warmup, dev):
 
 def time_kernel(fn, steps, warmup, dev):
     """Mean device time of fn(i), i = 0..steps-1; fn rotates over enough buffers that
-    one call finds none of its data in L2."""
+    one call finds none of its data in L2.  A device-side spin is queued ahead of the
+    timed calls: a kernel of a few tens of microseconds is shorter than the host's
+    work to launch it, so without the spin each event pair would also bracket the
+    device idling while the host prepares the launch.  With the device busy until
+    the host has queued every call, each pair brackets its kernel alone."""
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
     s, e = make_events(steps), make_events(steps)
+    torch.cuda._sleep(250_000 * steps)   # ~0.13 ms per timed call at 1.9 GHz
     for i in range(steps):
         s[i].record()
         fn(i)
