@@ -305,6 +305,25 @@ def active_weight_bytes(cfg, logits):
     return ids, ids * per_expert
 
 
+# Nominal dense tensor peaks of a B200: fp4 9 PFLOP/s against bf16 2.25 PFLOP/s.  With no
+# measured fp4 figure, the block-scaled fp4 peak is the measured bf16 peak times this ratio.
+FP4_OVER_BF16 = 9.0 / 2.25
+
+
+def w4a4_roofline(flops, weight_bytes, ms, pk):
+    """Roofline of a W4A4 layer: the slower of streaming its packed weights at the
+    measured HBM bandwidth and its flops at the block-scaled fp4 peak; `frac` is that
+    bound time over the measured time."""
+    mxf4 = pk["bf16"] * FP4_OVER_BF16
+    hbm_us = weight_bytes / pk["hbm"] / 1e3
+    mxf4_us = flops / mxf4 / 1e6
+    bound_us = max(hbm_us, mxf4_us)
+    return {"bound": "hbm" if hbm_us >= mxf4_us else "mxf4", "hbm_us": hbm_us, "mxf4_us": mxf4_us,
+            "mxf4_peak_tflops": mxf4,
+            "mxf4_peak_source": f"{pk['source']} bf16 x {FP4_OVER_BF16:g} (nominal dense fp4 / bf16)",
+            "bound_us": bound_us, "frac": bound_us / (ms * 1e3)}
+
+
 def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3):
     r = time_layer(L, cfg, mode, steps, warmup, dev)
     ms = statistics.mean(r["step_ms"])
@@ -328,6 +347,8 @@ def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3):
                     "frac_hbm": dn_w / st["down"] / 1e6 / pk["hbm"],
                     "tflops": fl / 3 / st["down"] / 1e9,
                     "frac_bf16": fl / 3 / st["down"] / 1e9 / pk["bf16"]}
+    if mode == 1:   # W4A4
+        line["roofline"] = w4a4_roofline(fl, wbytes, ms, pk)
     return line
 
 
