@@ -25,16 +25,20 @@ def _check(logits, k):
     assert np.all(np.abs(w - ref["w"]) <= 1e-6 * np.abs(ref["w"]) + 1e-7)
 
 
+# Shapes at the routing's limits (top-8 of 256 experts, top-1 of a few) and a token
+# count off the 8-token chunk boundary on either side of 256 pairs.
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (5, 4, 2), (63, 8, 3), (64, 32, 4), (65, 33, 4),
-                                   (200, 256, 8), (1000, 128, 4), (130, 7, 7)])
+                                   (200, 256, 8), (1000, 128, 4), (130, 7, 7), (32, 256, 8),
+                                   (256, 32, 1), (1, 256, 8), (257, 4, 1), (33, 256, 8)])
 def test_route_small(T, E, k):
     g = torch.Generator().manual_seed(T * 1000 + E)
     logits = torch.randn(T, E, generator=g)
     _check(logits, k)
 
 
-def test_route_ties_and_infinities():
-    T, E, k = 70, 16, 4
+@pytest.mark.parametrize("T", [70, 60])
+def test_route_ties_and_infinities(T):
+    E, k = 16, 4
     logits = torch.zeros(T, E)
     logits[1::3, 5] = 1.0
     logits[2::5, [3, 9, 12]] = 2.0
