@@ -435,8 +435,10 @@ int ring_grid(int64_t n_chunks, int sm_count) {
     return static_cast<int>(n_chunks < cap ? (n_chunks < 1 ? 1 : n_chunks) : cap);
 }
 
-// Opt the kernel in to the ring's dynamic shared memory (once per process; the
-// device is the same for every call of this library's process-wide cache).
+// Opt the kernel in to the ring's dynamic shared memory.  The attribute belongs to
+// the current device's context, so it is set before every launch (a host-side call
+// of about a microsecond) rather than cached, which stays right when the caller
+// switches devices.
 template <class K>
 cudaError_t set_ring_smem(K kern) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemBytes);
