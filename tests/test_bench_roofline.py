@@ -1,6 +1,9 @@
-"""bench.py's roofline arithmetic for the W4A4 layer, on CPU: the bound is the slower
-of streaming the packed expert weights at the HBM bandwidth and the layer's flops at
-the block-scaled fp4 peak (measured bf16 peak x the nominal fp4/bf16 ratio 4)."""
+"""bench.py's roofline pieces, on CPU.  The W4A4 layer's bound is the slower of
+streaming the packed expert weights at the HBM bandwidth and the layer's flops at the
+block-scaled fp4 peak (measured bf16 peak x the nominal fp4/bf16 ratio 4).  A DRAM
+traffic figure is reported only while the kernel sources hash to the value recorded
+with its ncu capture."""
+import json
 import os
 import sys
 
@@ -34,3 +37,24 @@ def test_flop_heavy_layer_is_mxf4_bound():
     assert r["bound"] == "mxf4"
     assert r["bound_us"] == pytest.approx(1e15 / (4 * 1640.9e12) * 1e6)
     assert 0 < r["frac"] < 1
+
+
+def test_traffic_is_reported_only_for_the_captured_source(monkeypatch, tmp_path):
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"k|w": {"dram_bytes_per_launch": 123.0, "source_sha256_16": "a" * 16}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "a" * 16)
+    assert bench.traffic_record("k", "w") == 123.0
+    assert bench.traffic_record("k", "other") is None          # not captured
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "b" * 16)
+    assert bench.traffic_record("k", "w") is None              # kernel source changed since
+
+
+def test_committed_traffic_record_is_well_formed():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    for key, r in recs.items():
+        kernel, workload = key.split("|")
+        assert r["dram_bytes_per_launch"] == r["dram_read_bytes"] + r["dram_write_bytes"]
+        assert len(r["source_sha256_16"]) == 16 and "ncu" in r["command"]
