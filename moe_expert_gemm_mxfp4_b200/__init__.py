@@ -44,10 +44,41 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need(t, dtype, shape, name):
-    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
-        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
-                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+def _need(t, name, dtype=None, shape=None):
+    """Raise unless `t` is a contiguous tensor of this dtype and shape.  The library
+    takes raw pointers: a strided view or a wrongly sized operand has to stop here,
+    not inside a kernel."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+
+
+def _on_current_device(**tensors):
+    """Raise unless every given tensor (None = absent) lives on the current CUDA device,
+    the one the library launches on: a host tensor would reach a kernel as a bad
+    address."""
+    cur = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA tensor, got one on {t.device}")
+        cur = torch.cuda.current_device() if cur is None else cur
+        if t.device.index != cur:
+            raise ValueError(f"{name}: on {t.device}, but the library launches on the current "
+                             f"device cuda:{cur}")
+
+
+def _need_dims(t, name, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim}-D, got shape {tuple(t.shape)}")
 
 
 def _empty(shape, dtype, like):
@@ -56,13 +87,18 @@ def _empty(shape, dtype, like):
 
 def mxfp4_quantize(x: torch.Tensor, rule: int = SCALE_FLOOR, codes=None, scales=None, stream=None):
     """x bf16/fp32 [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [rows, cols/32])."""
-    lib = _lib.load()
-    if x.dim() != 2:
-        raise ValueError("x must be 2-D")
+    _need_dims(x, "x", 2)
     R, C = x.shape
     dt = {torch.bfloat16: _lib.IN_BF16, torch.float32: _lib.IN_F32}.get(x.dtype)
     if dt is None:
-        raise ValueError("x must be bf16 or fp32")
+        raise ValueError(f"x: expected dtype bf16 or fp32, got {x.dtype}")
+    _need(x, "x")
+    if codes is not None:
+        _need(codes, "codes", torch.uint8, (R, C // 2))
+    if scales is not None:
+        _need(scales, "scales", torch.uint8, (R, C // 32))
+    _on_current_device(x=x, codes=codes, scales=scales)
+    lib = _lib.load()
     codes = _empty((R, C // 2), torch.uint8, x) if codes is None else codes
     scales = _empty((R, C // 32), torch.uint8, x) if scales is None else scales
     _lib.check("mxfp4_quantize", lib.mxfp4_quantize(_p(x), dt, R, C, _p(codes), _p(scales),
@@ -72,9 +108,15 @@ def mxfp4_quantize(x: torch.Tensor, rule: int = SCALE_FLOOR, codes=None, scales=
 
 def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, out=None, stream=None):
     """codes uint8 [rows, cols/2] + scales uint8 [rows, cols/32] -> bf16 [rows, cols]."""
-    lib = _lib.load()
+    _need_dims(codes, "codes", 2)
     R, half = codes.shape
     C = 2 * half
+    _need(codes, "codes", torch.uint8)
+    _need(scales, "scales", torch.uint8, (R, C // 32))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (R, C))
+    _on_current_device(codes=codes, scales=scales, out=out)
+    lib = _lib.load()
     out = _empty((R, C), torch.bfloat16, codes) if out is None else out
     _lib.check("mxfp4_dequantize", lib.mxfp4_dequantize(_p(codes), _p(scales), R, C, _p(out),
                                                         _stream(stream)))
@@ -88,9 +130,19 @@ def mxfp4_gemm_workspace_size(M, K, N, mode=W4A16) -> int:
 def mxfp4_gemm(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, mode: int = W4A16,
                out=None, ws=None, stream=None):
     """y bf16 [M, N] = x bf16 [M, K] . dequant(W)^T, W codes [N, K/2] + scales [N, K/32]."""
-    lib = _lib.load()
+    _need_dims(x, "x", 2)
+    _need_dims(w_codes, "w_codes", 2)
     M, K = x.shape
     N = w_codes.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(w_codes, "w_codes", torch.uint8, (N, K // 2))
+    _need(w_scales, "w_scales", torch.uint8, (N, K // 32))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (M, N))
+    if ws is not None:
+        _need(ws, "ws")
+    _on_current_device(x=x, w_codes=w_codes, w_scales=w_scales, out=out, ws=ws)
+    lib = _lib.load()
     out = _empty((M, N), torch.bfloat16, x) if out is None else out
     need = mxfp4_gemm_workspace_size(M, K, N, mode)
     if ws is None and need:
@@ -109,6 +161,11 @@ def moe_mxfp4_route(logits: torch.Tensor, top_k: int, ws=None, stream=None):
     """Top-k routing + expert-sorted permutation; returns a dict of device tensors
     ids [T, k] i32, weights [T, k] f32, counts [E] i32, offsets [E+1] i32,
     perm [T*k] i32, inv [T*k] i32."""
+    _need_dims(logits, "logits", 2)
+    _need(logits, "logits", torch.float32)
+    if ws is not None:
+        _need(ws, "ws")
+    _on_current_device(logits=logits, ws=ws)
     lib = _lib.load()
     T, E = logits.shape
     P = T * top_k
@@ -127,6 +184,30 @@ def moe_mxfp4_route(logits: torch.Tensor, top_k: int, ws=None, stream=None):
     return out
 
 
+def _check_moe_operands(x, logits, w13_codes, w13_scales, w2_codes, w2_scales, out):
+    """Shapes of one MoE layer's operands, from x [T, H], logits [T, E] and the
+    gate/up codes [E, 2I, H/2]; returns (T, H, E, I)."""
+    _need_dims(x, "x", 2)
+    _need_dims(logits, "logits", 2)
+    _need_dims(w13_codes, "w13_codes", 3)
+    T, H = x.shape
+    E = logits.shape[1]
+    if w13_codes.shape[1] % 2:
+        raise ValueError(f"w13_codes: expected [E, 2I, H/2], got {tuple(w13_codes.shape)}")
+    I = w13_codes.shape[1] // 2
+    _need(x, "x", torch.bfloat16)
+    _need(logits, "logits", torch.float32, (T, E))
+    _need(w13_codes, "w13_codes", torch.uint8, (E, 2 * I, H // 2))
+    _need(w13_scales, "w13_scales", torch.uint8, (E, 2 * I, H // 32))
+    _need(w2_codes, "w2_codes", torch.uint8, (E, H, I // 2))
+    _need(w2_scales, "w2_scales", torch.uint8, (E, H, I // 32))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (T, H))
+    _on_current_device(x=x, logits=logits, w13_codes=w13_codes, w13_scales=w13_scales,
+                       w2_codes=w2_codes, w2_scales=w2_scales, out=out)
+    return T, H, E, I
+
+
 def moe_mxfp4_workspace_size(T, H, I, E, top_k, mode=W4A16) -> int:
     return int(_lib.load().moe_mxfp4_workspace_size(T, H, I, E, top_k, int(mode)))
 
@@ -136,10 +217,11 @@ def moe_mxfp4_mlp(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13_codes, 
     """One MoE expert-MLP layer with MXFP4 expert weights (see include/mxfp4.h).
     x bf16 [T, H]; logits f32 [T, E]; w13 codes [E, 2I, H/2] + scales [E, 2I, H/32];
     w2 codes [E, H, I/2] + scales [E, H, I/32] -> out bf16 [T, H]."""
+    T, H, E, I = _check_moe_operands(x, logits, w13_codes, w13_scales, w2_codes, w2_scales, out)
+    if ws is not None:
+        _need(ws, "ws")
+        _on_current_device(ws=ws)
     lib = _lib.load()
-    T, H = x.shape
-    E = logits.shape[1]
-    I = w13_codes.shape[1] // 2
     out = _empty((T, H), torch.bfloat16, x) if out is None else out
     need = moe_mxfp4_workspace_size(T, H, I, E, top_k, mode)
     ws = _empty((need,), torch.uint8, x) if ws is None else ws
@@ -157,10 +239,8 @@ def moe_mxfp4_mlp_noalloc(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13
     under memory pressure).  Its scratch is a fixed 16 MiB array inside the library,
     shared by all calls: calls that overlap on the GPU race on it.  ``out`` is the
     caller's; pass it to keep this call allocation-free on the Python side too."""
+    T, H, E, I = _check_moe_operands(x, logits, w13_codes, w13_scales, w2_codes, w2_scales, out)
     lib = _lib.load()
-    T, H = x.shape
-    E = logits.shape[1]
-    I = w13_codes.shape[1] // 2
     out = _empty((T, H), torch.bfloat16, x) if out is None else out
     _lib.check("moe_mxfp4_mlp_noalloc", lib.moe_mxfp4_mlp_noalloc(
         _p(x), T, H, _p(logits), E, top_k, _p(w13_codes), _p(w13_scales), I, _p(w2_codes),
