@@ -55,15 +55,30 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+def nvsmi_device_id(props) -> str:
+    """The identifier nvidia-smi -i needs for a CUDA device, from its torch properties.
+
+    A CUDA device index is logical (it counts only the devices CUDA_VISIBLE_DEVICES
+    leaves visible), while nvidia-smi numbers every GPU of the machine, so the index
+    can name another GPU.  The device UUID (else its PCI bus id) names the same GPU
+    in both."""
+    uuid = getattr(props, "uuid", None)
+    if uuid:
+        u = str(uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """nvidia-smi clock / throttle-reason samples during the timed region (read-only
+    queries of the GPU given by its nvidia-smi identifier, see nvsmi_device_id)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
         self.proc = None
         self.path = None
 
@@ -220,35 +235,62 @@ def time_layer(L, cfg, mode, steps, warmup, dev, world=1, trace=True):
 
 
 def time_e2e(L, cfg, mode, steps, warmup, dev):
-    """Same layer through the public API with host buffers: pinned H2D of x and
-    the router logits, the call, D2H of the output -- all inside the timing."""
+    """Same layer through the public API with host buffers: every step copies its x
+    and router logits from pinned host memory to the device, runs the layer and copies
+    the output back to pinned host memory, all inside the timing.  Device inputs and
+    outputs are double-buffered so that one step's copies overlap another step's layer:
+    H2D on one copy stream, D2H on another, the layer on the compute stream, ordered by
+    events (a step's inputs land before its layer; a buffer is refilled only after the
+    layer that read it, and an output buffer is rewritten only after its copy back).
+    Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
     import moe_expert_gemm_mxfp4_b200 as mx
     T = L["x"].shape[0]
     hx = L["x"].pin_memory()
     hl = L["logits"].pin_memory()
-    hout = torch.empty((T, cfg.H), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(hx, device=dev)
-    ld = torch.empty_like(hl, device=dev)
-    out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    hout = [torch.empty((T, cfg.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(hx, device=dev) for _ in range(2)]
+    ld = [torch.empty_like(hl, device=dev) for _ in range(2)]
+    out = [torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     ws = torch.empty((mx.moe_mxfp4_workspace_size(T, cfg.H, cfg.I, cfg.E, cfg.top_k, mode),),
                      dtype=torch.uint8, device=dev)
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    landed = [ev() for _ in range(2)]
+    consumed = [ev() for _ in range(2)]
+    fetched = [ev() for _ in range(2)]
+    used = [False, False]
 
-    def one():
-        xd.copy_(hx, non_blocking=True)
-        ld.copy_(hl, non_blocking=True)
-        mx.moe_mxfp4_mlp(xd, ld, cfg.top_k, *L["w"], mode=mode, out=out, ws=ws)
-        hout.copy_(out, non_blocking=True)
+    def step(i):
+        b = i & 1
+        with torch.cuda.stream(up):
+            if used[b]:
+                up.wait_event(consumed[b])          # layer i-2 has read buffer b
+            xd[b].copy_(hx, non_blocking=True)
+            ld[b].copy_(hl, non_blocking=True)
+            landed[b].record(up)
+        comp.wait_event(landed[b])
+        if used[b]:
+            comp.wait_event(fetched[b])             # out[b] of step i-2 is back on the host
+        mx.moe_mxfp4_mlp(xd[b], ld[b], cfg.top_k, *L["w"], mode=mode, out=out[b], ws=ws)
+        consumed[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(consumed[b])
+            hout[b].copy_(out[b], non_blocking=True)
+            fetched[b].record(down)
+        used[b] = True
 
-    for _ in range(warmup):
-        one()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
-    a, b = make_events(2)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(up)
+    for i in range(steps):
+        step(warmup + i)
+    down.wait_event(fetched[(warmup + steps - 1) & 1])
+    z.record(down)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps, hx.numel() * 2 + hl.numel() * 4, hout.numel() * 2
+    return a.elapsed_time(z) / steps, hx.numel() * 2 + hl.numel() * 4, hout[0].numel() * 2
 
 
 def time_kernel(fn, steps, warmup, dev):
@@ -305,26 +347,58 @@ def active_weight_bytes(cfg, logits):
     return ids, ids * per_expert
 
 
-# Nominal dense tensor peaks of a B200: fp4 9 PFLOP/s against bf16 2.25 PFLOP/s.  With no
-# measured fp4 figure, the block-scaled fp4 peak is the measured bf16 peak times this ratio.
+# Nominal dense tensor peaks of a B200: fp4 9 PFLOP/s against bf16 2.25 PFLOP/s, the
+# ratio used only when the live probe below has not run.
 FP4_OVER_BF16 = 9.0 / 2.25
 
 
-def w4a4_roofline(flops, weight_bytes, ms, pk):
+def measure_mma_rates(dev, iters=36000, reps=3):
+    """Tensor-pipe rates of the library's two MMA kinds on this GPU, from its rate probe
+    (one CTA per SM, back-to-back M = 128, N = 256 MMAs on random operands; ~10 ms per
+    launch): best of `reps` launches each, in TFLOP/s, and their ratio mxf4 / f16."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    out = {}
+    for kind, name in ((0, "f16"), (1, "mxf4")):
+        mx.mxfp4_selftest_mma_rate(kind, 64)          # warm-up
+        best = 0.0
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fl = mx.mxfp4_selftest_mma_rate(kind, iters)
+            b.record()
+            torch.cuda.synchronize()
+            best = max(best, fl / a.elapsed_time(b) / 1e9)
+        out[name + "_tflops"] = best
+    assert mx.mxfp4_get_device_status() == 0
+    out["mxf4_over_f16"] = out["mxf4_tflops"] / out["f16_tflops"]
+    return out
+
+
+def mxf4_peak(pk, rates=None):
+    """Block-scaled fp4 (kind::mxf4) peak for the W4A4 roofline: the measured bf16 peak
+    times the mxf4 / f16 rate ratio the probe measured on this GPU (else the nominal 4)."""
+    if rates:
+        return (pk["bf16"] * rates["mxf4_over_f16"],
+                f"{pk['source']} bf16 x {rates['mxf4_over_f16']:.3f} (mxf4 / f16 tensor-pipe rate "
+                f"ratio measured by the library's probe: {rates['mxf4_tflops']:.0f} / "
+                f"{rates['f16_tflops']:.0f} TFLOP/s)")
+    return pk["bf16"] * FP4_OVER_BF16, f"{pk['source']} bf16 x {FP4_OVER_BF16:g} (nominal dense fp4 / bf16)"
+
+
+def w4a4_roofline(flops, weight_bytes, ms, pk, rates=None):
     """Roofline of a W4A4 layer: the slower of streaming its packed weights at the
     measured HBM bandwidth and its flops at the block-scaled fp4 peak; `frac` is that
     bound time over the measured time."""
-    mxf4 = pk["bf16"] * FP4_OVER_BF16
+    mxf4, src = mxf4_peak(pk, rates)
     hbm_us = weight_bytes / pk["hbm"] / 1e3
     mxf4_us = flops / mxf4 / 1e6
     bound_us = max(hbm_us, mxf4_us)
     return {"bound": "hbm" if hbm_us >= mxf4_us else "mxf4", "hbm_us": hbm_us, "mxf4_us": mxf4_us,
-            "mxf4_peak_tflops": mxf4,
-            "mxf4_peak_source": f"{pk['source']} bf16 x {FP4_OVER_BF16:g} (nominal dense fp4 / bf16)",
+            "mxf4_peak_tflops": mxf4, "mxf4_peak_source": src,
             "bound_us": bound_us, "frac": bound_us / (ms * 1e3)}
 
 
-def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3):
+def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3, rates=None):
     r = time_layer(L, cfg, mode, steps, warmup, dev)
     ms = statistics.mean(r["step_ms"])
     fl = layer_flops(cfg.T, cfg.top_k, cfg.H, cfg.I)
@@ -348,7 +422,7 @@ def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3):
                     "tflops": fl / 3 / st["down"] / 1e9,
                     "frac_bf16": fl / 3 / st["down"] / 1e9 / pk["bf16"]}
     if mode == 1:   # W4A4
-        line["roofline"] = w4a4_roofline(fl, wbytes, ms, pk)
+        line["roofline"] = w4a4_roofline(fl, wbytes, ms, pk, rates)
     return line
 
 
@@ -356,6 +430,8 @@ def breakdown(dev, pk):
     import moe_expert_gemm_mxfp4_b200 as mx
     from moe_expert_gemm_mxfp4_b200 import inputs
     bd = {"quant": bench_quant(dev, pk)}
+    rates = measure_mma_rates(dev)
+    bd["mma_probe"] = rates
     cfg = inputs.MOE_CONFIGS["moe_decode"]
     L = gpu_layer(cfg, dev)
     bd["moe_decode"] = bench_moe_line("moe_decode", cfg, L, mx.W4A16, dev, pk, steps=20)
@@ -363,7 +439,7 @@ def breakdown(dev, pk):
     cfg = inputs.MOE_CONFIGS["moe_120b"]
     L = gpu_layer(cfg, dev)
     bd["moe_120b_w4a16"] = bench_moe_line("moe_120b", cfg, L, mx.W4A16, dev, pk)
-    bd["moe_120b_w4a4"] = bench_moe_line("moe_120b", cfg, L, mx.W4A4, dev, pk)
+    bd["moe_120b_w4a4"] = bench_moe_line("moe_120b", cfg, L, mx.W4A4, dev, pk, rates=rates)
     del L
     torch.cuda.empty_cache()
     return bd
@@ -547,7 +623,7 @@ def main():
         cfg = dataclasses.replace(cfg, T=args.tokens)
     L = gpu_layer(cfg, dev)
 
-    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler = ClockSampler(nvsmi_device_id(torch.cuda.get_device_properties(dev)))
     sampler.start()
     r = time_layer(L, cfg, mx.W4A16, args.steps, args.warmup, dev, world=world)
     clocks = sampler.stop()

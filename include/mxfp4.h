@@ -78,7 +78,11 @@ typedef enum { MXFP4_W4A16 = 0, MXFP4_W4A4 = 1 } mxfp4_mode;
  * scales uint8 [rows, cols/32].  Per 32-element block: amax, E8M0 scale (rule),
  * E2M1 round-to-nearest-even of |v|/2^s saturating at 6, input sign bit copied
  * (-0 gives code 8); a block containing Inf/NaN gets S = 0xFF and zero codes.
- * Requires cols % 32 == 0.  Bit-exact: exactly one correct output exists. */
+ * Requires cols % 32 == 0.  Bit-exact: exactly one correct output exists.
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI GPT-OSS ...", section "What MXFP4 Is"
+ * (E2M1 elements with a 1/2/1 bit split; 32-element blocks share one scale), and
+ * otomatix.tech, the E2M1 sentence.  The scale encoding, scale exponent rule,
+ * rounding and packing are readings (listed above and in the encoding notes). */
 MXFP4_API mxfp4_status mxfp4_quantize(const void* x, mxfp4_in_dtype dt, int64_t rows, int64_t cols,
                             uint8_t* codes, uint8_t* scales, mxfp4_scale_rule rule,
                             void* stream);
@@ -86,7 +90,10 @@ MXFP4_API mxfp4_status mxfp4_quantize(const void* x, mxfp4_in_dtype dt, int64_t 
 /* ---------------------------------------------------------------- dequantize
  * codes uint8 [rows, cols/2] + scales uint8 [rows, cols/32] -> out bf16 [rows, cols].
  * value = code_value * 2^(S-127) rounded once to bf16 (exact except overflow to
- * Inf); S = 0xFF gives NaN.  Requires cols % 32 == 0. */
+ * Inf); S = 0xFF gives NaN.  Requires cols % 32 == 0.
+ * Source: the same section "What MXFP4 Is" (value = E2M1 element x block scale);
+ * section "Native Support in transformers" names the bf16 form this produces (the
+ * fallback at about four times the memory). */
 MXFP4_API mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
                               int64_t rows, int64_t cols, void* out_bf16, void* stream);
 
@@ -96,7 +103,11 @@ MXFP4_API mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* sca
  * Requires K % 64 == 0 and K <= 7680 (the block scales of a 128-row weight tile
  * are staged whole in shared memory); any M >= 1, N >= 1.  Workspace: W4A16 needs none
  * (ws may be NULL); W4A4 needs mxfp4_gemm_workspace_size() bytes (x quantized to
- * MXFP4: codes and block scales). */
+ * MXFP4: codes and block scales).
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI GPT-OSS ...", section "MXFP4 4-Bit
+ * Quantization" (MXFP4 weights multiplied by specialized kernels without a bf16 copy)
+ * and "What MXFP4 Is"; W4A4 reads "the same quantised math" as quantizing the
+ * activations with mxfp4_quantize's FLOOR rule. */
 MXFP4_API mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K,
                         const uint8_t* w_codes, const uint8_t* w_scales, int64_t N,
                         void* y_bf16, mxfp4_mode mode, void* ws, size_t ws_bytes,
@@ -111,8 +122,12 @@ MXFP4_API size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp
  * sum), perm int32 [P] (perm[offsets[e] + r] = the r-th pair routed to e in
  * ascending p) and inv int32 [P] (inv[perm[i]] = i), P = T*top_k.
  * Requires 1 <= top_k <= min(E, 8), E <= 256, T*top_k < 2^31.
+ * A NaN logit ranks below every number (-inf included), NaNs among themselves by id.
  * ids/counts/offsets/perm/inv are bit-exact; weights match an fp64 softmax to
- * ~1e-6 relative. */
+ * ~1e-6 relative.
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI GPT-OSS ...", section "Zero-Build Kernels
+ * from the Hub" (the MoE layer runs as a MegaBlocks MoE kernel, which routes each
+ * token to its top experts); the ordering, tie rule and softmax scope are readings. */
 MXFP4_API mxfp4_status moe_mxfp4_route(const float* router_logits, int64_t T, int64_t E, int32_t top_k,
                              int32_t* ids, float* weights, int32_t* counts, int32_t* offsets,
                              int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
@@ -131,7 +146,12 @@ MXFP4_API size_t moe_mxfp4_route_workspace_size(int64_t T, int64_t E, int32_t to
  * scales uint8 [E, 2I, H/32]; w2 codes uint8 [E, H, I/2] + scales [E, H, I/32];
  * out bf16 [T, H].  Requires H % 64 == 0, I % 64 == 0, H, I <= 7680, 1 <= top_k <= min(E, 8),
  * E <= 256, T*top_k < 2^31.  ws must hold moe_mxfp4_workspace_size() bytes
- * (routing tables and the per-pair activations h / y). */
+ * (routing tables and the per-pair activations h / y).
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI GPT-OSS ...", sections "Zero-Build
+ * Kernels from the Hub" (the MoE expert MLP as one MegaBlocks MoE kernel) and "MXFP4
+ * 4-Bit Quantization" (its expert weights in MXFP4); the gated-SiLU expert MLP,
+ * gate/up row split and weighted combine are readings of "h = SiLU(gate) * up;
+ * out = sum of weight x down(h)". */
 MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,
                            const float* router_logits, int64_t E, int32_t top_k,
                            const uint8_t* w13_codes, const uint8_t* w13_scales, int64_t I,
@@ -197,6 +217,16 @@ MXFP4_API const char* mxfp4_status_string(mxfp4_status s);
  * stays usable.  Returns MXFP4_OK once launched (read the outcome with
  * mxfp4_get_device_status), or MXFP4_ERR_ARCH / MXFP4_ERR_CUDA. */
 MXFP4_API mxfp4_status mxfp4_selftest_wait_timeout(void* stream);
+/* Tensor-pipe rate probe (no counterpart in the pages; it supplies the roofline
+ * denominator of the block-scaled MMA, which no library figure gives for this box).
+ * Launches one CTA per SM on `stream`; each issues iters x 4 back-to-back
+ * tcgen05.mma of M = 128, N = 256 from shared memory: kind = 0 is kind::f16 (bf16
+ * operands, K = 16 per MMA), kind = 1 is kind::mxf4.block_scale (E2M1 operands with
+ * E8M0 scales, K = 64 per MMA).  Operands are pseudo-random finite values.  *flops
+ * receives the launch's multiply-add count x 2; time the launch with events on
+ * `stream` and divide.  Requires 1 <= iters <= 2^20.  Errors as the other entry
+ * points (a completion wait that runs out records MXFP4_ERR_TIMEOUT). */
+MXFP4_API mxfp4_status mxfp4_selftest_mma_rate(int32_t kind, int32_t iters, double* flops, void* stream);
 
 #ifdef __cplusplus
 }

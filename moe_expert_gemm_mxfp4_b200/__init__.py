@@ -25,7 +25,7 @@ __all__ = [
     "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_gemm_workspace_size",
     "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
     "moe_mxfp4_workspace_size", "moe_mxfp4_mlp_noalloc", "mxfp4_get_device_status",
-    "mxfp4_selftest_wait_timeout", "mxfp4_set_trace_events",
+    "mxfp4_selftest_wait_timeout", "mxfp4_selftest_mma_rate", "mxfp4_set_trace_events",
     "Mxfp4Error", "Mxfp4LibraryMissing",
     "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
 ]
@@ -258,6 +258,17 @@ def mxfp4_selftest_wait_timeout(stream=None):
     gives up after the library's wait limit and records MXFP4_ERR_TIMEOUT."""
     _lib.check("mxfp4_selftest_wait_timeout",
                _lib.load().mxfp4_selftest_wait_timeout(_stream(stream)))
+
+
+def mxfp4_selftest_mma_rate(kind: int, iters: int, stream=None) -> float:
+    """Launch the tensor-pipe rate probe (kind 0: kind::f16 bf16 MMAs, 1: block-scaled
+    kind::mxf4 MMAs; one CTA per SM, iters x 4 MMAs of M = 128, N = 256 each) on the
+    stream and return the launch's flop count.  Time it with CUDA events."""
+    flops = ctypes.c_double(0.0)
+    _lib.check("mxfp4_selftest_mma_rate",
+               _lib.load().mxfp4_selftest_mma_rate(int(kind), int(iters), ctypes.byref(flops),
+                                                   _stream(stream)))
+    return flops.value
 
 
 _trace_keepalive = None

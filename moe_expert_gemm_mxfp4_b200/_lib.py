@@ -60,6 +60,7 @@ _SIGS = {
                                              ctypes.c_int, _vp]),
     "mxfp4_get_device_status": (ctypes.c_int, [_vp]),
     "mxfp4_selftest_wait_timeout": (ctypes.c_int, [_vp]),
+    "mxfp4_selftest_mma_rate": (ctypes.c_int, [_i32, _i32, ctypes.POINTER(ctypes.c_double), _vp]),
     "mxfp4_set_trace_events": (None, [_vp, ctypes.c_int]),
     "mxfp4_last_cuda_error": (ctypes.c_int, []),
     "mxfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),

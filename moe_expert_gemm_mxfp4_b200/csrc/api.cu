@@ -234,6 +234,17 @@ mxfp4_status mxfp4_selftest_wait_timeout(void* stream) {
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
+mxfp4_status mxfp4_selftest_mma_rate(int32_t kind, int32_t iters, double* flops, void* stream) {
+    if ((kind != 0 && kind != 1) || iters <= 0 || iters > (1 << 20) || !flops) return MXFP4_ERR_INVALID_ARG;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    *flops = mx::selftest_mma_flops(kind, iters, d->sm_count);
+    cudaError_t e = mx::launch_selftest_mma_rate(kind, iters, d->sm_count, d->status,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
 void mxfp4_set_trace_events(void* const* events, int n_events) {
     tl_trace_events = n_events > 0 ? events : nullptr;
     tl_trace_n = n_events > 0 ? n_events : 0;
@@ -550,8 +561,13 @@ mxfp4_status moe_mxfp4_mlp_noalloc(const void* x_bf16, int64_t T, int64_t H,
     if ((st = device_info(&d)) != MXFP4_OK) return st;
     void* ws = nullptr;
     if ((st = noalloc_scratch(&ws)) != MXFP4_OK) return st;
-    // every scratch byte the layer reads is written earlier in the same call, so the
-    // previous call's leftovers need no clearing
+    // Every scratch byte a result depends on is written earlier in the same call, so
+    // the previous call's leftovers need no clearing.  The one exception is read but
+    // never used: in W4A4, the GEMM stages a token tile's scales with one bulk copy of
+    // the 16-byte-aligned range that covers them, which takes in up to 16 bytes past
+    // the end of an activation-scale array (the tail the carving keeps readable); no
+    // kernel writes that tail, and the scale bytes past a tile's rows never reach an
+    // MMA, so whatever an earlier call left there cannot change the output.
     return moe_mxfp4_mlp(x_bf16, T, H, router_logits, E, top_k, w13_codes, w13_scales, I,
                          w2_codes, w2_scales, out_bf16, mode, ws, MXFP4_NOALLOC_SCRATCH_BYTES,
                          stream);

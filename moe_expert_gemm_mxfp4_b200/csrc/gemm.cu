@@ -11,9 +11,9 @@
 // 4.40 performance upgrades for OpenAI GPT-OSS ...", sections "What MXFP4 Is"
 // and "Zero-Build Kernels from the Hub").
 //
-// Work tile: 128 weight rows (the MMA's M side) x TT token tiles of NT rows
-// (the N side).  The weights are dequantized once per 64-wide K stage and used
-// by TT MMAs, so TT = 2 halves the dequant work and the weight traffic per flop.
+// Work tile: 128 weight rows (the MMA's M side) x NT token rows (the N side).
+// The weights are dequantized once per 64-wide K stage.  (The engine is written
+// for TT token tiles per weight tile; every launch uses TT = 1.)
 //
 // Data flow (one persistent CTA per SM, 16 warps):
 //   warp 0        codes producer: per tile the block scales of its 128 rows
@@ -596,10 +596,7 @@ cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap
         int sc, sa, smem;
         if (ring_depths<192, 1>(a.K, &sc, &sa, &smem)) return launch_cfg<192, 1, MODE>(tw, tx, a, grid, stream);
     }
-    if (tt == 2) {   // two token tiles per weight tile when their rings fit this K
-        int sc, sa, smem;
-        if (ring_depths<128, 2>(a.K, &sc, &sa, &smem)) return launch_cfg<128, 2, MODE>(tw, tx, a, grid, stream);
-    }
+    (void)tt;   // one token tile per weight tile in every configuration
     return launch_cfg<128, 1, MODE>(tw, tx, a, grid, stream);
 }
 

@@ -44,6 +44,9 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int64
                               int64_t cols, void* out, int sm_count, unsigned* status,
                               cudaStream_t stream);
 cudaError_t launch_selftest_wait_timeout(unsigned* status, cudaStream_t stream);
+double selftest_mma_flops(int kind, int iters, int sm_count);
+cudaError_t launch_selftest_mma_rate(int kind, int iters, int sm_count, unsigned* status,
+                                     cudaStream_t stream);
 size_t route_tmp_bytes(int64_t T, int64_t E, int top_k);
 cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, int32_t* ids,
                          float* weights, int32_t* counts, int32_t* offsets, int32_t* perm,

@@ -12,8 +12,9 @@
 // token, expert and output vector gets its own warp or thread, so that a decode
 // step (tens of tokens) costs a few microseconds per launch.
 //   route_topk     one warp per token: top-k and softmax; per CTA (a chunk of
-//                  8 tokens) the per-expert pair counts and each pair's rank
-//                  among the chunk's pairs of its expert;
+//                  8 tokens, at most 64 pairs in two warps) the per-expert pair
+//                  counts and each pair's rank among the chunk's pairs of its
+//                  expert, from warp match masks and population counts;
 //   route_scan     one CTA per expert: exclusive scan of its chunk counts ->
 //                  per-chunk base ranks, and the expert's total;
 //   route_scatter  offsets (exclusive scan over experts, recomputed per CTA in
@@ -33,16 +34,25 @@ constexpr int kMaxExperts = 256;
 
 namespace {
 
+// Expert order: larger logit first, lower expert id among equal logits; a NaN logit
+// ranks below every number (-inf included), NaNs among themselves by id.  This is a
+// strict total order, so every lane of the butterfly below ends with the same pick.
 __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
-    return v > bv || (v == bv && id < bid);
+    const bool vn = v != v, bn = bv != bv;
+    if (vn != bn) return bn;
+    if (!vn && v != bv) return v > bv;
+    return id < bid;
 }
 
 __global__ void __launch_bounds__(kRouteThreads)
 route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ ids,
                   float* __restrict__ weights, int32_t* __restrict__ chunk_counts,
                   int32_t* __restrict__ local_rank) {
+    static_assert(kTokPerChunk * kMaxTopK <= 64, "a chunk's pairs must fit in warps 0 and 1");
     __shared__ int32_t s_ids[kTokPerChunk * kMaxTopK];
+    __shared__ int32_t s_cnt[kMaxExperts];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
     const int t0 = blockIdx.x * kTokPerChunk;
     const int ntok = min(kTokPerChunk, T - t0);
     const int t = t0 + wid;
@@ -107,19 +117,26 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t
         }
     }
     __syncthreads();
-    // the chunk's pairs i = 0 .. ntok*k - 1 in ascending p: counts and stable ranks
+    // The chunk's pairs i = 0 .. ntok*k - 1 (ascending p, at most 64) sit one per
+    // thread of warps 0 and 1.  Within a warp, the lanes holding the same expert are
+    // one match mask: a pair's rank is the number of matching lanes below it, the
+    // warp's count of that expert the mask's population.  Warp 1 adds warp 0's count.
     const int npairs = ntok * k;
-    if (static_cast<int>(threadIdx.x) < npairs) {
-        const int e = s_ids[threadIdx.x];
-        int r = 0;
-        for (int i = 0; i < static_cast<int>(threadIdx.x); ++i) r += s_ids[i] == e;
-        local_rank[static_cast<int64_t>(t0) * k + threadIdx.x] = r;
-    }
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int c = 0;
-        for (int i = 0; i < npairs; ++i) c += s_ids[i] == e;
-        chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = c;
-    }
+    const int i = threadIdx.x;
+    const bool valid = i < npairs;
+    const int e = valid ? s_ids[i] : kMaxExperts + lane;   // out-of-range ids match no pair
+    uint32_t m = 0;
+    if (wid < 2) m = __match_any_sync(0xFFFFFFFFu, e);
+    const uint32_t below = m & ((1u << lane) - 1u);
+    const bool leader = below == 0;
+    if (wid == 0 && valid && leader) s_cnt[e] = __popc(m);
+    __syncthreads();
+    if (valid) local_rank[static_cast<int64_t>(t0) * k + i] = __popc(below) + (wid == 1 ? s_cnt[e] : 0);
+    __syncthreads();   // every rank has read warp 0's counts
+    if (wid == 1 && valid && leader) s_cnt[e] += __popc(m);
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += blockDim.x)
+        chunk_counts[static_cast<int64_t>(blockIdx.x) * E + x] = s_cnt[x];
 }
 
 // Block-wide exclusive scan of one int per thread (blockDim.x == kRouteThreads);

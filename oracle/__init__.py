@@ -169,7 +169,9 @@ def route(logits: np.ndarray, top_k: int):
 
     Readings (the pages only say the MoE layer routes tokens to experts):
       * experts ordered by (logit descending, expert id ascending), exact fp32
-        comparison -- ties go to the lower expert id;
+        comparison -- ties go to the lower expert id; a NaN logit ranks below
+        every number (-inf included), NaNs among themselves by id (numpy's sort
+        places NaN last, and the stable sort keeps ids ascending);
       * w_tj = exp(l_tj - l_t0) / sum_i exp(l_ti - l_t0) over the k selected
         logits, in fp64;
       * pair p = t * k + j; counts[e] = #pairs routed to e; offsets = exclusive

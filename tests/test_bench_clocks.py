@@ -20,7 +20,7 @@ class _DoneProcess:
 def _read(tmp_path, lines):
     path = tmp_path / "clocks.csv"
     path.write_text("".join(l + "\n" for l in lines))
-    cs = bench.ClockSampler(0)
+    cs = bench.ClockSampler("GPU-00000000-0000-0000-0000-000000000000")
     cs.path, cs.proc = str(path), _DoneProcess()
     out = cs.stop()
     assert not path.exists()          # the sampler removes its file
@@ -48,3 +48,32 @@ def test_slowdown_reasons_are_reported(tmp_path):
 
 def test_no_samples_reads_as_none(tmp_path):
     assert _read(tmp_path, []) is None
+
+
+class _Props:
+    def __init__(self, uuid=None, domain=0, bus=0x3B, device=0):
+        self.uuid, self.pci_domain_id, self.pci_bus_id, self.pci_device_id = uuid, domain, bus, device
+
+
+def test_sampler_names_the_gpu_by_uuid_not_by_logical_index(monkeypatch):
+    # With CUDA_VISIBLE_DEVICES=5, CUDA device 0 is the machine's GPU 5: nvidia-smi must
+    # be given that GPU's UUID, never the logical index 0.
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "5")
+    u = "4b1f6a2e-1c3d-4e5f-8a9b-0c1d2e3f4a5b"
+    assert bench.nvsmi_device_id(_Props(uuid=u)) == "GPU-" + u
+    assert bench.nvsmi_device_id(_Props(uuid="GPU-" + u)) == "GPU-" + u
+    assert bench.nvsmi_device_id(_Props(uuid=None, bus=0x9A)) == "00000000:9a:00.0"
+    seen = {}
+
+    class _Popen:
+        def __init__(self, cmd, **kw):
+            seen["cmd"] = cmd
+
+    monkeypatch.setattr(bench.subprocess, "Popen", _Popen)
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    cs = bench.ClockSampler(bench.nvsmi_device_id(_Props(uuid=u)))
+    cs.start()
+    os.unlink(cs.path)
+    cmd = seen["cmd"]
+    assert cmd[cmd.index("-i") + 1] == "GPU-" + u
+    assert not any(a.startswith(("-lgc", "-ac", "-pm", "-rgc", "-r")) for a in cmd)   # read-only query

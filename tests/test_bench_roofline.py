@@ -58,3 +58,15 @@ def test_committed_traffic_record_is_well_formed():
         kernel, workload = key.split("|")
         assert r["dram_bytes_per_launch"] == r["dram_read_bytes"] + r["dram_write_bytes"]
         assert len(r["source_sha256_16"]) == 16 and "ncu" in r["command"]
+
+
+def test_measured_mma_ratio_sets_the_mxf4_peak():
+    # the probe's mxf4 / f16 tensor-pipe rate ratio replaces the nominal 4
+    rates = {"f16_tflops": 2100.0, "mxf4_tflops": 8358.0, "mxf4_over_f16": 8358.0 / 2100.0}
+    peak, src = bench.mxf4_peak(PK, rates)
+    assert peak == pytest.approx(1640.9 * 8358.0 / 2100.0)
+    assert "probe" in src
+    r = bench.w4a4_roofline(1e15, 1e6, 1000.0, PK, rates)
+    assert r["mxf4_peak_tflops"] == pytest.approx(peak)
+    assert r["bound_us"] == pytest.approx(1e15 / (peak * 1e12) * 1e6)
+    assert bench.mxf4_peak(PK, None)[0] == pytest.approx(4 * 1640.9)

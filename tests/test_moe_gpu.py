@@ -104,3 +104,30 @@ def test_moe_120b_w4a4_sampled(l120):
 def test_moe_small_w4a4_all_tokens():
     L = Layer(_small(64, 256, 192, 8, 2, seed=5))
     assert_close_tol(L.gpu(mx.W4A4), L.ref(mode="w4a4"), what="small W4A4")
+
+
+def _avg_rows(T, E, k):
+    return -(-T * k // E)
+
+
+# Token tiles of 32 and 64 rows (experts averaging 17-32 and 33-64 routed rows) with
+# both fused epilogues (SwiGLU, weighted), in W4A16 and W4A4, every token compared.
+@pytest.mark.parametrize("mode", [mx.W4A16, mx.W4A4])
+@pytest.mark.parametrize("T,H,I,nt", [(160, 384, 320, 32), (256, 256, 192, 32),
+                                      (400, 320, 256, 64), (512, 256, 384, 64)])
+def test_moe_mid_token_tiles_all_tokens(mode, T, H, I, nt):
+    E, k = 32, 4
+    assert nt // 2 < _avg_rows(T, E, k) <= nt
+    L = Layer(_small(T, H, I, E, k, seed=T + H))
+    ref = L.ref(mode="w4a16" if mode == mx.W4A16 else "w4a4")
+    assert_close_tol(L.gpu(mode), ref, what=f"moe T={T} E={E} (NT={nt}) mode={mode}")
+
+
+def test_moe_decode_batch_256_tokens_full_size():
+    """A 256-token decode batch of the gpt-oss-20b-shaped layer (experts average 32
+    routed rows, so the 32-row token tile), every token compared, W4A16 and W4A4."""
+    cfg = inputs.MOE_CONFIGS["moe_decode"]
+    L = Layer(cfg, T=256)
+    assert 16 < _avg_rows(256, cfg.E, cfg.top_k) <= 32
+    assert_close_tol(L.gpu(mx.W4A16), L.ref(), what="decode T=256 W4A16")
+    assert_close_tol(L.gpu(mx.W4A4), L.ref(mode="w4a4"), what="decode T=256 W4A4")

@@ -334,6 +334,32 @@ def test_route_bruteforce():
         assert np.all(flat[seg] == e) and np.all(np.diff(seg) > 0)
 
 
+def test_route_nan_logits_rank_below_every_number():
+    # Reading: a NaN router logit ranks below every number, -inf included; NaNs
+    # among themselves by expert id.  Brute force with that key.
+    g = torch.Generator().manual_seed(22)
+    T, E, k = 12, 9, 4
+    logits = torch.randn(T, E, generator=g).numpy()
+    logits[0, [1, 4]] = np.nan
+    logits[1, :] = np.nan                      # all NaN: ids 0..k-1, NaN weights
+    logits[2, [0, 2, 3, 5, 6, 7, 8]] = np.nan  # two numbers, then NaNs by id
+    logits[3, [2, 6]] = -np.inf
+    logits[3, [0, 1, 3, 4, 5]] = np.nan        # -inf ranks above NaN
+    r = oracle.route(logits, k)
+
+    def key(t, e):
+        v = float(logits[t, e])
+        return (1, 0.0, e) if math.isnan(v) else (0, -v, e)
+
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: key(t, e))[:k]
+        assert list(r["ids"][t]) == order, t
+    assert list(r["ids"][2][:2]) == [1, 4] and np.isnan(r["w"][2]).all()
+    assert sorted(r["ids"][3][:2]) == [7, 8] and list(r["ids"][3][2:]) == [2, 6]   # -inf above NaN
+    assert np.isnan(r["w"][1]).all()
+    assert np.all(np.isfinite(r["w"][4:]))
+
+
 # ----------------------------------------------------------------- GEMM
 
 def test_gemm_bruteforce():

@@ -22,7 +22,9 @@ def _check(logits, k):
     assert np.array_equal(r["perm"].cpu().numpy(), ref["perm"])
     assert np.array_equal(r["inv"].cpu().numpy(), ref["inv"])
     w = r["weights"].cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(w - ref["w"]) <= 1e-6 * np.abs(ref["w"]) + 1e-7)
+    nan = np.isnan(ref["w"])
+    assert np.array_equal(np.isnan(w), nan)
+    assert np.all(np.abs(w - ref["w"])[~nan] <= 1e-6 * np.abs(ref["w"][~nan]) + 1e-7)
 
 
 # Shapes at the routing's limits (top-8 of 256 experts, top-1 of a few) and a token
@@ -53,3 +55,19 @@ def test_route_workloads(name):
     cfg = inputs.MOE_CONFIGS[name]
     _, logits = inputs.moe_activations(cfg)
     _check(logits, cfg.top_k)
+
+
+def test_route_nan_logits():
+    # NaN logits rank below every number (-inf included), NaNs among themselves by id;
+    # a token that has to select a NaN gets NaN weights on every slot
+    T, E, k = 45, 40, 4
+    g = torch.Generator().manual_seed(7)
+    logits = torch.randn(T, E, generator=g)
+    logits[0, [1, 4, 33]] = float("nan")
+    logits[1, :] = float("nan")
+    logits[2, :] = float("nan")
+    logits[2, [5, 39]] = 1.0
+    logits[3, 10:] = float("-inf")
+    logits[3, :10] = float("nan")
+    logits[9::4, 0] = float("nan")
+    _check(logits, k)
