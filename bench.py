@@ -426,10 +426,33 @@ def bench_moe_line(name, cfg, L, mode, dev, pk, steps=10, warmup=3, rates=None):
     return line
 
 
+def bench_route_project(dev, steps=20, warmup=5):
+    """Routing from the tokens (router projection fused with top-k, moe_mxfp4_route_project)
+    against routing from precomputed logits (moe_mxfp4_route), per call, at the decode
+    and prefill workloads' shapes.  Router weights bf16 [E, H] ~ N(0, 1/H)."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    out = {}
+    for name in ("moe_decode", "moe_prefill"):
+        cfg = inputs.MOE_CONFIGS[name]
+        x, logits = inputs.moe_activations(cfg)
+        x, logits, w = x.to(dev), logits.to(dev), inputs.router_weights(cfg).to(dev)
+        ws = torch.empty((mx.moe_mxfp4_route_workspace_size(cfg.T, cfg.E, cfg.top_k),), dtype=torch.uint8,
+                         device=dev)
+        tp = time_kernel(lambda i: mx.moe_mxfp4_route_project(x, w, cfg.top_k, ws=ws), steps, warmup, dev)
+        tr = time_kernel(lambda i: mx.moe_mxfp4_route(logits, cfg.top_k, ws=ws), steps, warmup, dev)
+        proj_flops = 2.0 * cfg.T * cfg.E * cfg.H
+        out[name] = {"T": cfg.T, "E": cfg.E, "H": cfg.H, "route_project_us": tp * 1e3,
+                     "route_from_logits_us": tr * 1e3, "projection_tflops": proj_flops / tp / 1e9}
+    assert mx.mxfp4_get_device_status() == 0
+    return out
+
+
 def breakdown(dev, pk):
     import moe_expert_gemm_mxfp4_b200 as mx
     from moe_expert_gemm_mxfp4_b200 import inputs
     bd = {"quant": bench_quant(dev, pk)}
+    bd["route_project"] = bench_route_project(dev)
     rates = measure_mma_rates(dev)
     bd["mma_probe"] = rates
     cfg = inputs.MOE_CONFIGS["moe_decode"]

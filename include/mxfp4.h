@@ -132,6 +132,25 @@ MXFP4_API mxfp4_status moe_mxfp4_route(const float* router_logits, int64_t T, in
                              int32_t* ids, float* weights, int32_t* counts, int32_t* offsets,
                              int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
                              void* stream);
+/* ---------------------------------------------------------------- router projection + routing
+ * The same routing computed from the tokens themselves: logits[t, e] = x[t] . W_r[e]
+ * (x bf16 [T, H], router weights bf16 [E, H], products exact, fp32 accumulation on
+ * the tensor cores), then exactly the ordering, softmax and tables of
+ * moe_mxfp4_route applied to those fp32 logits, in the same launch: the logits are
+ * not written to memory unless `logits_out` (fp32 [T, E], may be NULL) asks for a
+ * copy.  Same outputs, workspace (moe_mxfp4_route_workspace_size) and errors as
+ * moe_mxfp4_route; requires H % 64 == 0.  The logits agree with an fp64 dot product
+ * to within fp32 accumulation error (H * 2^-24 * sum |x * w|), so ids can differ
+ * from an fp64 router's only where two logits are that close.
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI
+ * GPT-OSS ...", section "Zero-Build Kernels from the Hub" (the MoE kernel's routing;
+ * a top-k kernel); the bias-free linear router is a reading. */
+MXFP4_API mxfp4_status moe_mxfp4_route_project(const void* x_bf16, int64_t T, int64_t H,
+                                               const void* w_router_bf16, int64_t E, int32_t top_k,
+                                               int32_t* ids, float* weights, int32_t* counts,
+                                               int32_t* offsets, int32_t* perm, int32_t* inv,
+                                               float* logits_out, void* ws, size_t ws_bytes,
+                                               void* stream);
 /* Scratch bytes moe_mxfp4_route needs in `ws` (per-chunk counts and ranks). */
 MXFP4_API size_t moe_mxfp4_route_workspace_size(int64_t T, int64_t E, int32_t top_k);
 
@@ -161,6 +180,43 @@ MXFP4_API mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H,
 MXFP4_API size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k,
                                 mxfp4_mode mode);
 
+/* ---------------------------------------------------------------- the layer's parts, for composition
+ * The MoE layer above is route -> experts -> combine.  These entry points expose the
+ * parts after routing, so that a caller can move the expert-sorted rows between
+ * GPUs in between (expert parallelism: each GPU runs the experts it holds on the
+ * rows routed to them from every GPU, then sends the results back).
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI
+ * GPT-OSS ...", section "Expert Parallelism (EP)" (MoE experts distributed across
+ * GPUs); the split into these parts is this library's design.
+ *
+ * mxfp4_gather_rows: dst row i = src row (idx[i] / div) for i < n, rows of row_bytes
+ * bytes (a multiple of 4); src [n_src rows], idx int32 [n], dst [n rows].  With
+ * div = top_k and idx = the routing's perm, it gathers token rows into expert-sorted
+ * order.  An index whose row is outside src leaves its dst row unwritten and
+ * records MXFP4_ERR_INVALID_ARG in the device status word. */
+MXFP4_API mxfp4_status mxfp4_gather_rows(const void* src, int64_t n_src, int64_t row_bytes,
+                                         const int32_t* idx, int64_t n, int32_t div, void* dst,
+                                         void* stream);
+/* moe_mxfp4_experts: the experts of one layer on rows already grouped by expert:
+ * x_sorted bf16 [P, H] with expert e's rows at offsets[e] .. offsets[e+1] (int32
+ * [E+1], device), routing weight row_w fp32 [P] ->
+ *   h = bf16(SiLU(x W13[e][0:I]^T) * (x W13[e][I:2I]^T)),  y = row_w * (h W2[e]^T)
+ * into y_sorted fp32 [P, H] (W4A4: x and h MXFP4-quantized first, as in the layer).
+ * Weights and requirements as moe_mxfp4_mlp; offsets must be non-decreasing with
+ * offsets[0] = 0 and offsets[E] = P.  ws: moe_mxfp4_experts_workspace_size() bytes. */
+MXFP4_API mxfp4_status moe_mxfp4_experts(const void* x_sorted_bf16, int64_t P, int64_t H,
+                                         const int32_t* offsets, int64_t E, const uint8_t* w13_codes,
+                                         const uint8_t* w13_scales, int64_t I, const uint8_t* w2_codes,
+                                         const uint8_t* w2_scales, const float* row_w, float* y_sorted,
+                                         mxfp4_mode mode, void* ws, size_t ws_bytes, void* stream);
+MXFP4_API size_t moe_mxfp4_experts_workspace_size(int64_t P, int64_t H, int64_t I, int64_t E,
+                                                  mxfp4_mode mode);
+/* moe_mxfp4_combine: out[t] = bf16( sum_j y_sorted[inv[t*top_k + j]] ) summed in fp32 in
+ * slot order j = 0 .. top_k-1 (deterministic); y_sorted fp32 [*, H], inv int32
+ * [T*top_k], out bf16 [T, H].  Requires H % 8 == 0, top_k <= 8. */
+MXFP4_API mxfp4_status moe_mxfp4_combine(const float* y_sorted, const int32_t* inv, int64_t T,
+                                         int32_t top_k, int64_t H, void* out_bf16, void* stream);
+
 /* ---------------------------------------------------------------- allocation-free MoE layer
  * Not a step of the method: the pages have no counterpart of this entry point.
  *
@@ -172,9 +228,9 @@ MXFP4_API size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64
  * scratch is one fixed array of MXFP4_NOALLOC_SCRATCH_BYTES in device memory, set
  * aside on every GPU that loads the library until the process exits.
  *   - Limit: calls whose moe_mxfp4_workspace_size(...) exceeds
- *     MXFP4_NOALLOC_SCRATCH_BYTES return MXFP4_ERR_WORKSPACE (with H = I = 2880 and
- *     32 experts that is up to 724 token-expert pairs, T * top_k, in W4A16 and 808
- *     in W4A4: decode batches).
+ *     MXFP4_NOALLOC_SCRATCH_BYTES return MXFP4_ERR_WORKSPACE (with H = I = 2880,
+ *     32 experts and top-4 that is up to 724 token-expert pairs, T * top_k, in W4A16
+ *     and 808 in W4A4: decode batches).
  *   - The first call on each device looks up the array's device address (a host-side
  *     query, no allocation); make that first call before any stream capture.
  *   - All calls share the one array: calls that overlap on the GPU (other streams, or

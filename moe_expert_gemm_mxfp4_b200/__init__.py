@@ -26,6 +26,8 @@ __all__ = [
     "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
     "moe_mxfp4_workspace_size", "moe_mxfp4_mlp_noalloc", "mxfp4_get_device_status",
     "mxfp4_selftest_wait_timeout", "mxfp4_selftest_mma_rate", "mxfp4_set_trace_events",
+    "moe_mxfp4_route_project", "mxfp4_gather_rows", "moe_mxfp4_experts",
+    "moe_mxfp4_experts_workspace_size", "moe_mxfp4_combine",
     "Mxfp4Error", "Mxfp4LibraryMissing",
     "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
 ]
@@ -181,6 +183,112 @@ def moe_mxfp4_route(logits: torch.Tensor, top_k: int, ws=None, stream=None):
         _p(logits), T, E, top_k, _p(out["ids"]), _p(out["weights"]), _p(out["counts"]),
         _p(out["offsets"]), _p(out["perm"]), _p(out["inv"]), _p(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def moe_mxfp4_route_project(x: torch.Tensor, w_router: torch.Tensor, top_k: int, logits_out: bool = False,
+                            ws=None, stream=None):
+    """Router projection fused with top-k routing: logits = x . w_router^T (bf16
+    x [T, H], bf16 w_router [E, H], fp32 accumulation), then the routing of
+    ``moe_mxfp4_route``.  Returns the same dict, plus ``logits`` (fp32 [T, E]) when
+    ``logits_out`` is set."""
+    _need_dims(x, "x", 2)
+    _need_dims(w_router, "w_router", 2)
+    _need(x, "x", torch.bfloat16)
+    T, H = x.shape
+    _need(w_router, "w_router", torch.bfloat16, (w_router.shape[0], H))
+    if ws is not None:
+        _need(ws, "ws")
+    _on_current_device(x=x, w_router=w_router, ws=ws)
+    lib = _lib.load()
+    E = w_router.shape[0]
+    P = T * top_k
+    out = dict(ids=_empty((T, top_k), torch.int32, x),
+               weights=_empty((T, top_k), torch.float32, x),
+               counts=_empty((E,), torch.int32, x),
+               offsets=_empty((E + 1,), torch.int32, x),
+               perm=_empty((P,), torch.int32, x),
+               inv=_empty((P,), torch.int32, x))
+    if logits_out:
+        out["logits"] = _empty((T, E), torch.float32, x)
+    need = moe_mxfp4_route_workspace_size(T, E, top_k)
+    ws = _empty((need,), torch.uint8, x) if ws is None else ws
+    _lib.check("moe_mxfp4_route_project", lib.moe_mxfp4_route_project(
+        _p(x), T, H, _p(w_router), E, top_k, _p(out["ids"]), _p(out["weights"]), _p(out["counts"]),
+        _p(out["offsets"]), _p(out["perm"]), _p(out["inv"]), _p(out["logits"]) if logits_out else None,
+        _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def mxfp4_gather_rows(src: torch.Tensor, idx: torch.Tensor, div: int = 1, out=None, stream=None):
+    """out[i] = src[idx[i] // div] (rows of a 2-D contiguous tensor; row bytes a
+    multiple of 4); idx int32 [n]."""
+    _need_dims(src, "src", 2)
+    _need(src, "src")
+    _need(idx, "idx", torch.int32)
+    n = idx.numel()
+    if out is None:
+        out = _empty((n, src.shape[1]), src.dtype, src)
+    else:
+        _need(out, "out", src.dtype, (n, src.shape[1]))
+    _on_current_device(src=src, idx=idx, out=out)
+    _lib.check("mxfp4_gather_rows", _lib.load().mxfp4_gather_rows(
+        _p(src), src.shape[0], src.shape[1] * src.element_size(), _p(idx), n, int(div), _p(out),
+        _stream(stream)))
+    return out
+
+
+def moe_mxfp4_experts_workspace_size(P, H, I, E, mode=W4A16) -> int:
+    return int(_lib.load().moe_mxfp4_experts_workspace_size(P, H, I, E, int(mode)))
+
+
+def moe_mxfp4_experts(x_sorted: torch.Tensor, offsets: torch.Tensor, row_w: torch.Tensor, w13_codes,
+                      w13_scales, w2_codes, w2_scales, mode: int = W4A16, out=None, ws=None, stream=None):
+    """The experts on expert-grouped rows: x_sorted bf16 [P, H], offsets int32 [E+1],
+    row_w fp32 [P] -> y_sorted fp32 [P, H] = row_w * down(SwiGLU(gate_up(x)))."""
+    _need_dims(x_sorted, "x_sorted", 2)
+    _need(x_sorted, "x_sorted", torch.bfloat16)
+    P, H = x_sorted.shape
+    _need_dims(w13_codes, "w13_codes", 3)
+    E, twoI, _ = w13_codes.shape
+    I = twoI // 2
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(row_w, "row_w", torch.float32, (P,))
+    _need(w13_codes, "w13_codes", torch.uint8, (E, 2 * I, H // 2))
+    _need(w13_scales, "w13_scales", torch.uint8, (E, 2 * I, H // 32))
+    _need(w2_codes, "w2_codes", torch.uint8, (E, H, I // 2))
+    _need(w2_scales, "w2_scales", torch.uint8, (E, H, I // 32))
+    if out is None:
+        out = _empty((P, H), torch.float32, x_sorted)
+    else:
+        _need(out, "out", torch.float32, (P, H))
+    need = moe_mxfp4_experts_workspace_size(P, H, I, E, mode)
+    if ws is None:
+        ws = _empty((max(need, 16),), torch.uint8, x_sorted)
+    else:
+        _need(ws, "ws")
+    _on_current_device(x_sorted=x_sorted, offsets=offsets, row_w=row_w, w13_codes=w13_codes,
+                       w13_scales=w13_scales, w2_codes=w2_codes, w2_scales=w2_scales, out=out, ws=ws)
+    _lib.check("moe_mxfp4_experts", _lib.load().moe_mxfp4_experts(
+        _p(x_sorted), P, H, _p(offsets), E, _p(w13_codes), _p(w13_scales), I, _p(w2_codes), _p(w2_scales),
+        _p(row_w), _p(out), int(mode), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def moe_mxfp4_combine(y_sorted: torch.Tensor, inv: torch.Tensor, top_k: int, out=None, stream=None):
+    """out[t] = bf16(sum_j y_sorted[inv[t*k + j]]) in slot order; y_sorted fp32 [*, H]."""
+    _need_dims(y_sorted, "y_sorted", 2)
+    _need(y_sorted, "y_sorted", torch.float32)
+    _need(inv, "inv", torch.int32)
+    H = y_sorted.shape[1]
+    T = inv.numel() // top_k
+    if out is None:
+        out = _empty((T, H), torch.bfloat16, y_sorted)
+    else:
+        _need(out, "out", torch.bfloat16, (T, H))
+    _on_current_device(y_sorted=y_sorted, inv=inv, out=out)
+    _lib.check("moe_mxfp4_combine", _lib.load().moe_mxfp4_combine(
+        _p(y_sorted), _p(inv), T, top_k, H, _p(out), _stream(stream)))
     return out
 
 

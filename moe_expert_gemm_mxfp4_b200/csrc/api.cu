@@ -206,6 +206,127 @@ int gemm_grid(const DeviceInfo* d, int64_t tile_bound) {
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
+// Operands of the experts' two grouped GEMMs (gate/up + SwiGLU, then down x the
+// routing weight), all device memory.
+struct ExpertsIO {
+    const void* x_rows;       // W4A16: bf16 activation rows in expert-sorted order
+    int64_t x_rows_n;         // rows of x_rows
+    const uint8_t* xs_codes;  // W4A4: sorted activation rows as MXFP4 (codes, scales + 16 B)
+    const uint8_t* xs_scales;
+    const int32_t* offsets;   // [E + 1] sorted-row offsets of the experts
+    const float* row_w;       // [P] routing weight of every sorted row
+    void* h;                  // bf16 [P, I]
+    uint8_t* hq_codes;        // W4A4: h as MXFP4
+    uint8_t* hq_scales;
+    void* y_sorted;           // fp32 [P, H] out
+};
+
+void trace_mark(int i, cudaStream_t s);
+
+// The experts of one layer on their expert-sorted rows: h = bf16(SiLU(x W_g^T) * (x W_u^T)),
+// then y = w * (h W_2^T) in fp32 (W4A4: x and h quantized to MXFP4 first).
+mxfp4_status run_experts(DeviceInfo* d, int64_t P, int64_t H, int64_t I, int64_t E, mxfp4_mode mode,
+                         const uint8_t* w13_codes, const uint8_t* w13_scales, const uint8_t* w2_codes,
+                         const uint8_t* w2_scales, const ExpertsIO& io, cudaStream_t s) {
+    const bool a4 = mode == MXFP4_W4A4;
+    mxfp4_status st;
+    cudaError_t e;
+    // W4A16 with at most 32 rows per expert on average: the small-group (mma.sync) engine
+    const int nt_h = a4 ? 0 : mx::pick_token_tiling_hmma(P, E);
+    const bool small = nt_h > 0 && mx::hmma_fits_k(H) && mx::hmma_fits_k(I);
+    mx::TokenTiling tiling = a4 ? mx::pick_token_tiling_w4a4(P, E) : mx::pick_token_tiling(P, E);
+    if (small) tiling = {nt_h, 1};
+    const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
+    const int64_t tok_tiles = (P + tile_rows - 1) / tile_rows + E;
+
+    // gate/up projection with the SwiGLU epilogue -> h [P, I]
+    CUtensorMap tw, tx;
+    if ((st = encode_codes_map(&tw, w13_codes, H, 2 * I, E, a4 ? 16 : 64)) != MXFP4_OK) return st;
+    st = a4 ? encode_x4_map(&tx, io.xs_codes, H, P, tiling.nt)
+            : encode_act_map(&tx, io.x_rows, H, io.x_rows_n, tiling.nt);
+    if (st != MXFP4_OK) return st;
+    mx::GemmArgs a{};
+    a.w_scales = w13_scales;
+    a.x_scales = io.xs_scales;
+    a.offsets = io.offsets;
+    a.m_single = 0;
+    a.G = static_cast<int>(E);
+    a.K = static_cast<int>(H);
+    a.rows_w = static_cast<int>(2 * I);
+    a.I = static_cast<int>(I);
+    a.n_ftiles = static_cast<int>(I / 64);
+    a.out = io.h;
+    a.out_ld = I;
+    a.n_valid_feat = static_cast<int>(I);
+    a.row_w = nullptr;
+    a.status = d->status;
+    const int grid1 = gemm_grid(d, tok_tiles * a.n_ftiles);
+    e = a4      ? mx::launch_grouped_gemm_w4a4(mx::EPI_SWIGLU, tiling.nt, tw, tx, a, grid1, s)
+        : small ? mx::launch_grouped_gemm_hmma(mx::EPI_SWIGLU, tiling.nt, tw, tx, a, grid1, s)
+                : mx::launch_grouped_gemm(mx::EPI_SWIGLU, tiling, tw, tx, a, grid1, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+
+    trace_mark(2, s);
+    if (a4) {   // h to MXFP4 (FLOOR rule, blocks along I)
+        if ((e = mx::launch_quantize(io.h, 0, P, I, io.hq_codes, io.hq_scales, MXFP4_SCALE_FLOOR,
+                                     d->sm_count, d->status, s)) != cudaSuccess)
+            return cuda_fail(e);
+    }
+
+    // down projection, routing weight applied in fp32 -> y_sorted fp32 [P, H]
+    if ((st = encode_codes_map(&tw, w2_codes, I, H, E, 128)) != MXFP4_OK) return st;
+    st = a4 ? encode_x4_map(&tx, io.hq_codes, I, P, tiling.nt) : encode_act_map(&tx, io.h, I, P, tiling.nt);
+    if (st != MXFP4_OK) return st;
+    a.w_scales = w2_scales;
+    a.x_scales = io.hq_scales;
+    a.K = static_cast<int>(I);
+    a.rows_w = static_cast<int>(H);
+    a.I = 0;
+    a.n_ftiles = static_cast<int>((H + 127) / 128);
+    a.out = io.y_sorted;
+    a.out_ld = H;
+    a.n_valid_feat = static_cast<int>(H);
+    a.row_w = io.row_w;
+    const int grid2 = gemm_grid(d, tok_tiles * a.n_ftiles);
+    e = a4      ? mx::launch_grouped_gemm_w4a4(mx::EPI_WEIGHTED, tiling.nt, tw, tx, a, grid2, s)
+        : small ? mx::launch_grouped_gemm_hmma(mx::EPI_WEIGHTED, tiling.nt, tw, tx, a, grid2, s)
+                : mx::launch_grouped_gemm(mx::EPI_WEIGHTED, tiling, tw, tx, a, grid2, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    trace_mark(3, s);
+    return MXFP4_OK;
+}
+
+// Workspace of moe_mxfp4_experts: W4A4 sorted rows as MXFP4, h, W4A4 h as MXFP4.
+struct ExpertsWs {
+    uint8_t* xs_codes;
+    uint8_t* xs_scales;
+    void* h;
+    uint8_t* hq_codes;
+    uint8_t* hq_scales;
+    size_t bytes;
+};
+
+ExpertsWs carve_experts(void* base, int64_t P, int64_t H, int64_t I, int mode) {
+    ExpertsWs w{};
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        void* p = base ? static_cast<uint8_t*>(base) + off : nullptr;
+        off = align_up(off + n, 256);
+        return p;
+    };
+    if (mode == MXFP4_W4A4) {
+        w.xs_codes = static_cast<uint8_t*>(take(static_cast<size_t>(P) * H / 2));
+        w.xs_scales = static_cast<uint8_t*>(take(static_cast<size_t>(P) * H / 32 + 16));
+    }
+    w.h = take(static_cast<size_t>(P) * I * 2);
+    if (mode == MXFP4_W4A4) {
+        w.hq_codes = static_cast<uint8_t*>(take(static_cast<size_t>(P) * I / 2));
+        w.hq_scales = static_cast<uint8_t*>(take(static_cast<size_t>(P) * I / 32 + 16));
+    }
+    w.bytes = off;
+    return w;
+}
+
 }  // namespace
 
 extern "C" {
@@ -326,8 +447,11 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     mxfp4_status st = device_info(&d);
     if (st != MXFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const mx::TokenTiling tiling =
+    mx::TokenTiling tiling =
         mode == MXFP4_W4A4 ? mx::pick_token_tiling_w4a4(M, 1) : mx::pick_token_tiling(M, 1);
+    const int nt_h = mode == MXFP4_W4A4 ? 0 : mx::pick_token_tiling_hmma(M, 1);
+    const bool small = nt_h > 0 && mx::hmma_fits_k(K);   // at most 32 rows: the mma.sync engine
+    if (small) tiling = {nt_h, 1};
     CUtensorMap tw, tx;
     if ((st = encode_codes_map(&tw, w_codes, K, N, 1, 128)) != MXFP4_OK) return st;
     uint8_t* xq_codes = static_cast<uint8_t*>(ws);
@@ -361,8 +485,9 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     cudaError_t e = mode == MXFP4_W4A4
                         ? mx::launch_grouped_gemm_w4a4(mx::EPI_PLAIN, tiling.nt, tw, tx, a,
                                                        gemm_grid(d, tiles), s)
-                        : mx::launch_grouped_gemm(mx::EPI_PLAIN, tiling, tw, tx, a,
-                                                  gemm_grid(d, tiles), s);
+                    : small ? mx::launch_grouped_gemm_hmma(mx::EPI_PLAIN, tiling.nt, tw, tx, a, gemm_grid(d, tiles), s)
+                            : mx::launch_grouped_gemm(mx::EPI_PLAIN, tiling, tw, tx, a,
+                                                      gemm_grid(d, tiles), s);
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
@@ -394,8 +519,45 @@ mxfp4_status moe_mxfp4_route(const float* router_logits, int64_t T, int64_t E, i
     DeviceInfo* d = nullptr;
     if ((st = device_info(&d)) != MXFP4_OK) return st;
     cudaError_t e = mx::launch_route(router_logits, T, E, top_k, ids, weights, counts, offsets, perm,
-                                     inv, nullptr, ws, nullptr, 0, nullptr, nullptr, 0, nullptr,
+                                     inv, nullptr, nullptr, ws, nullptr, 0, nullptr, nullptr, 0, nullptr,
                                      d->sm_count, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+mxfp4_status moe_mxfp4_route_project(const void* x_bf16, int64_t T, int64_t H, const void* w_router_bf16,
+                                     int64_t E, int32_t top_k, int32_t* ids, float* weights,
+                                     int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                                     float* logits_out, void* ws, size_t ws_bytes, void* stream) {
+    if (!x_bf16 || !w_router_bf16 || !ids || !weights || !counts || !offsets || !perm || !inv)
+        return MXFP4_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || E <= 0 || top_k <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (E > 256 || top_k > 8 || top_k > E) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (H % 64 != 0 || T * top_k >= (int64_t{1} << 31) || H >= (int64_t{1} << 31))
+        return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(w_router_bf16) || !aligned16(ids) || !aligned16(weights) ||
+        !aligned16(counts) || !aligned16(offsets) || !aligned16(perm) || !aligned16(inv) ||
+        (logits_out && !aligned16(logits_out)))
+        return MXFP4_ERR_MISALIGNED;
+    const size_t need = moe_mxfp4_route_workspace_size(T, E, top_k);
+    if (!ws || ws_bytes < need) return MXFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // x [T, H] in 128-token boxes; W_r [E, H] in one box of E rounded up to 16 rows
+    // (the rows past E are the TMA's zero fill)
+    CUtensorMap tx, tw;
+    if ((st = encode_act_map(&tx, x_bf16, H, T, 128)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tw, w_router_bf16, H, E, static_cast<int>((E + 15) / 16 * 16))) != MXFP4_OK)
+        return st;
+    int32_t *chunk_counts, *local_rank;
+    mx::route_tmp_split(ws, T, E, &chunk_counts, &local_rank);
+    cudaError_t e = mx::launch_route_project(tx, tw, T, H, E, top_k, ids, weights, chunk_counts,
+                                             local_rank, logits_out, d->status, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = mx::launch_route_finish(T, E, top_k, ids, weights, counts, offsets, perm, inv, nullptr, nullptr,
+                                ws, nullptr, 0, nullptr, nullptr, 0, nullptr, d->sm_count, s);
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
@@ -443,72 +605,31 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
                                      d->sm_count, d->status, s)) != cudaSuccess)
             return cuda_fail(e);
         e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets,
-                             w.perm, w.inv, w.w_sorted, w.route_tmp, w.xq_codes, H / 2, w.xs_codes,
-                             w.xq_scales, H / 32, w.xs_scales, d->sm_count, s);
+                             w.perm, w.inv, w.w_sorted, nullptr, w.route_tmp, w.xq_codes, H / 2,
+                             w.xs_codes, w.xq_scales, H / 32, w.xs_scales, d->sm_count, s);
     } else {
+        // W4A16: the routing's scatter also copies every token row to its expert-sorted
+        // position (one 16-byte vector per lane, all loads before the stores)
         e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets,
-                             w.perm, w.inv, w.w_sorted, w.route_tmp, x_bf16, H * 2, w.x_sorted,
+                             w.perm, w.inv, w.w_sorted, nullptr, w.route_tmp, x_bf16, H * 2, w.x_sorted,
                              nullptr, 0, nullptr, d->sm_count, s);
     }
     if (e != cudaSuccess) return cuda_fail(e);
 
     trace_mark(1, s);
-    const mx::TokenTiling tiling = a4 ? mx::pick_token_tiling_w4a4(P, E) : mx::pick_token_tiling(P, E);
-    const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
-    const int64_t tok_tiles = (P + tile_rows - 1) / tile_rows + E;
-
-    // gate/up projection with the SwiGLU epilogue -> h [P, I]
-    CUtensorMap tw, tx;
-    if ((st = encode_codes_map(&tw, w13_codes, H, 2 * I, E, a4 ? 16 : 64)) != MXFP4_OK) return st;
-    st = a4 ? encode_x4_map(&tx, w.xs_codes, H, P, tiling.nt)
-            : encode_act_map(&tx, w.x_sorted, H, P, tiling.nt);
-    if (st != MXFP4_OK) return st;
-    mx::GemmArgs a{};
-    a.w_scales = w13_scales;
-    a.x_scales = w.xs_scales;
-    a.offsets = w.offsets;
-    a.m_single = 0;
-    a.G = static_cast<int>(E);
-    a.K = static_cast<int>(H);
-    a.rows_w = static_cast<int>(2 * I);
-    a.I = static_cast<int>(I);
-    a.n_ftiles = static_cast<int>(I / 64);
-    a.out = w.h;
-    a.out_ld = I;
-    a.n_valid_feat = static_cast<int>(I);
-    a.row_w = nullptr;
-    a.status = d->status;
-    const int grid1 = gemm_grid(d, tok_tiles * a.n_ftiles);
-    e = a4 ? mx::launch_grouped_gemm_w4a4(mx::EPI_SWIGLU, tiling.nt, tw, tx, a, grid1, s)
-           : mx::launch_grouped_gemm(mx::EPI_SWIGLU, tiling, tw, tx, a, grid1, s);
-    if (e != cudaSuccess) return cuda_fail(e);
-
-    trace_mark(2, s);
-    if (a4) {   // h to MXFP4 (FLOOR rule, blocks along I)
-        if ((e = mx::launch_quantize(w.h, 0, P, I, w.hq_codes, w.hq_scales, MXFP4_SCALE_FLOOR,
-                                     d->sm_count, d->status, s)) != cudaSuccess)
-            return cuda_fail(e);
-    }
-
-    // down projection, routing weight applied in fp32 -> y_sorted fp32 [P, H]
-    if ((st = encode_codes_map(&tw, w2_codes, I, H, E, 128)) != MXFP4_OK) return st;
-    st = a4 ? encode_x4_map(&tx, w.hq_codes, I, P, tiling.nt)
-            : encode_act_map(&tx, w.h, I, P, tiling.nt);
-    if (st != MXFP4_OK) return st;
-    a.w_scales = w2_scales;
-    a.x_scales = w.hq_scales;
-    a.K = static_cast<int>(I);
-    a.rows_w = static_cast<int>(H);
-    a.I = 0;
-    a.n_ftiles = static_cast<int>((H + 127) / 128);
-    a.out = w.y_sorted;
-    a.out_ld = H;
-    a.n_valid_feat = static_cast<int>(H);
-    a.row_w = w.w_sorted;
-    const int grid2 = gemm_grid(d, tok_tiles * a.n_ftiles);
-    e = a4 ? mx::launch_grouped_gemm_w4a4(mx::EPI_WEIGHTED, tiling.nt, tw, tx, a, grid2, s)
-           : mx::launch_grouped_gemm(mx::EPI_WEIGHTED, tiling, tw, tx, a, grid2, s);
-    if (e != cudaSuccess) return cuda_fail(e);
+    ExpertsIO io{};
+    io.x_rows = w.x_sorted;
+    io.x_rows_n = P;
+    io.xs_codes = w.xs_codes;
+    io.xs_scales = w.xs_scales;
+    io.offsets = w.offsets;
+    io.row_w = w.w_sorted;
+    io.h = w.h;
+    io.hq_codes = w.hq_codes;
+    io.hq_scales = w.hq_scales;
+    io.y_sorted = w.y_sorted;
+    if ((st = run_experts(d, P, H, I, E, mode, w13_codes, w13_scales, w2_codes, w2_scales, io, s)) != MXFP4_OK)
+        return st;
 
     trace_mark(3, s);
     // deterministic combine in slot order
@@ -517,6 +638,84 @@ mxfp4_status moe_mxfp4_mlp(const void* x_bf16, int64_t T, int64_t H, const float
         return cuda_fail(e);
     trace_mark(4, s);
     return MXFP4_OK;
+}
+
+mxfp4_status mxfp4_gather_rows(const void* src, int64_t n_src, int64_t row_bytes, const int32_t* idx,
+                               int64_t n, int32_t div, void* dst, void* stream) {
+    if (!src || !idx || !dst) return MXFP4_ERR_INVALID_ARG;
+    if (n_src <= 0 || n <= 0 || row_bytes <= 0 || div <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (row_bytes % 4 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(src) || !aligned16(idx) || !aligned16(dst)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaError_t e = mx::launch_gather_rows(src, n_src, row_bytes, idx, n, div, dst, d->sm_count, d->status,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+size_t moe_mxfp4_experts_workspace_size(int64_t P, int64_t H, int64_t I, int64_t E, mxfp4_mode mode) {
+    (void)E;
+    if (P <= 0 || H <= 0 || I <= 0) return 0;
+    return carve_experts(nullptr, P, H, I, mode).bytes;
+}
+
+mxfp4_status moe_mxfp4_experts(const void* x_sorted_bf16, int64_t P, int64_t H, const int32_t* offsets,
+                               int64_t E, const uint8_t* w13_codes, const uint8_t* w13_scales, int64_t I,
+                               const uint8_t* w2_codes, const uint8_t* w2_scales, const float* row_w,
+                               float* y_sorted, mxfp4_mode mode, void* ws, size_t ws_bytes, void* stream) {
+    if (!x_sorted_bf16 || !offsets || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !row_w ||
+        !y_sorted)
+        return MXFP4_ERR_INVALID_ARG;
+    if (P <= 0 || H <= 0 || I <= 0 || E <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (mode != MXFP4_W4A16 && mode != MXFP4_W4A4) return MXFP4_ERR_INVALID_ARG;
+    if (E > 256 || P >= (int64_t{1} << 31)) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (H % 64 != 0 || I % 64 != 0) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (H > mx::max_gemm_k() || I > mx::max_gemm_k()) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (mode == MXFP4_W4A4 && (H > mx::max_gemm_k_w4a4() || I > mx::max_gemm_k_w4a4()))
+        return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_sorted_bf16) || !aligned16(offsets) || !aligned16(w13_codes) || !aligned16(w13_scales) ||
+        !aligned16(w2_codes) || !aligned16(w2_scales) || !aligned16(row_w) || !aligned16(y_sorted))
+        return MXFP4_ERR_MISALIGNED;
+    const size_t need = moe_mxfp4_experts_workspace_size(P, H, I, E, mode);
+    if (!ws || ws_bytes < need) return MXFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const ExpertsWs w = carve_experts(ws, P, H, I, mode);
+    if (mode == MXFP4_W4A4) {
+        cudaError_t e = mx::launch_quantize(x_sorted_bf16, 0, P, H, w.xs_codes, w.xs_scales, MXFP4_SCALE_FLOOR,
+                                            d->sm_count, d->status, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    ExpertsIO io{};
+    io.x_rows = x_sorted_bf16;
+    io.x_rows_n = P;
+    io.xs_codes = w.xs_codes;
+    io.xs_scales = w.xs_scales;
+    io.offsets = offsets;
+    io.row_w = row_w;
+    io.h = w.h;
+    io.hq_codes = w.hq_codes;
+    io.hq_scales = w.hq_scales;
+    io.y_sorted = y_sorted;
+    return run_experts(d, P, H, I, E, mode, w13_codes, w13_scales, w2_codes, w2_scales, io, s);
+}
+
+mxfp4_status moe_mxfp4_combine(const float* y_sorted, const int32_t* inv, int64_t T, int32_t top_k, int64_t H,
+                               void* out_bf16, void* stream) {
+    if (!y_sorted || !inv || !out_bf16) return MXFP4_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || top_k <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (top_k > 8 || H % 8 != 0 || T * top_k >= (int64_t{1} << 31)) return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(y_sorted) || !aligned16(inv) || !aligned16(out_bf16)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    mxfp4_status st = device_info(&d);
+    if (st != MXFP4_OK) return st;
+    cudaError_t e = mx::launch_combine(y_sorted, inv, T, top_k, H, out_bf16, d->sm_count,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
 }
 
 // ---------------------------------------------------------------- allocation-free MoE layer

@@ -589,9 +589,7 @@ cudaError_t launch_cfg(const CUtensorMap& tw, const CUtensorMap& tx, GemmArgs a,
 template <int MODE>
 cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap& tx,
                         const GemmArgs& a, int grid, cudaStream_t stream) {
-    if (nt == 16) return launch_cfg<16, 1, MODE>(tw, tx, a, grid, stream);
-    if (nt == 32) return launch_cfg<32, 1, MODE>(tw, tx, a, grid, stream);
-    if (nt == 64) return launch_cfg<64, 1, MODE>(tw, tx, a, grid, stream);
+    if (nt <= 64) return launch_cfg<64, 1, MODE>(tw, tx, a, grid, stream);
     if (nt == 192) {
         int sc, sa, smem;
         if (ring_depths<192, 1>(a.K, &sc, &sa, &smem)) return launch_cfg<192, 1, MODE>(tw, tx, a, grid, stream);
@@ -603,11 +601,10 @@ cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap
 }  // namespace
 
 // Token tiling for `rows` activation rows spread over `groups` groups: NT rows per
-// MMA (16..128) and TT token tiles per dequantized weight tile.
+// MMA (64, 128 or 192; groups averaging at most 32 rows go to the small-group
+// mma.sync engine of gemm_hmma.cu instead).
 TokenTiling pick_token_tiling(int64_t rows, int64_t groups) {
     const int64_t avg = (rows + groups - 1) / (groups > 0 ? groups : 1);
-    if (avg <= 16) return {16, 1};
-    if (avg <= 32) return {32, 1};
     if (avg <= 64) return {64, 1};
     // 192-row token tiles dequantize each weight tile once per 192 tokens instead of
     // 128 (the dequantize work bounds the large-batch GEMM), at the cost of a ragged
@@ -623,8 +620,7 @@ int64_t max_gemm_k() {
     int sc, sa, smem;
     while (ring_depths<128, 1>(static_cast<int>(k + 64), &sc, &sa, &smem) &&
            ring_depths<64, 1>(static_cast<int>(k + 64), &sc, &sa, &smem) &&
-           ring_depths<32, 1>(static_cast<int>(k + 64), &sc, &sa, &smem) &&
-           ring_depths<16, 1>(static_cast<int>(k + 64), &sc, &sa, &smem))
+           hmma_fits_k(k + 64))
         k += 64;
     return k;
 }

@@ -50,9 +50,23 @@ cudaError_t launch_selftest_mma_rate(int kind, int iters, int sm_count, unsigned
 size_t route_tmp_bytes(int64_t T, int64_t E, int top_k);
 cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, int32_t* ids,
                          float* weights, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv, float* w_sorted, void* tmp, const void* x,
+                         int32_t* inv, float* w_sorted, int32_t* row_tok, void* tmp, const void* x,
                          int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
                          void* xs_sorted, int sm_count, cudaStream_t stream);
+cudaError_t launch_route_finish(int64_t T, int64_t E, int top_k, const int32_t* ids, const float* weights,
+                                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                                float* w_sorted, int32_t* row_tok, void* tmp, const void* x,
+                                int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
+                                void* xs_sorted, int sm_count, cudaStream_t stream);
+void route_tmp_split(void* tmp, int64_t T, int64_t E, int32_t** chunk_counts, int32_t** local_rank);
+int route_project_smem_bytes(int64_t E);
+cudaError_t launch_route_project(const CUtensorMap& tmap_x, const CUtensorMap& tmap_w, int64_t T,
+                                 int64_t H, int64_t E, int top_k, int32_t* ids, float* weights,
+                                 int32_t* chunk_counts, int32_t* local_rank, float* logits_out,
+                                 unsigned* status, cudaStream_t stream);
+cudaError_t launch_gather_rows(const void* src, int64_t n_src, int64_t row_bytes, const int32_t* idx,
+                               int64_t n, int div, void* dst, int sm_count, unsigned* status,
+                               cudaStream_t stream);
 cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, int top_k,
                            int64_t H, void* out, int sm_count, cudaStream_t stream);
 TokenTiling pick_token_tiling(int64_t rows, int64_t groups);
@@ -60,6 +74,10 @@ int64_t max_gemm_k();   // largest contraction length the grouped GEMM accepts
 cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream);
+int pick_token_tiling_hmma(int64_t rows, int64_t groups);   // 16, 32, or 0 (groups too large)
+bool hmma_fits_k(int64_t K);
+cudaError_t launch_grouped_gemm_hmma(int mode, int nt, const CUtensorMap& tmap_w, const CUtensorMap& tmap_x,
+                                     const GemmArgs& args, int grid, cudaStream_t stream);
 int64_t max_gemm_k_w4a4();   // largest contraction length the W4A4 engine accepts
 TokenTiling pick_token_tiling_w4a4(int64_t rows, int64_t groups);
 cudaError_t launch_grouped_gemm_w4a4(int mode, int nt, const CUtensorMap& tmap_w,

@@ -284,6 +284,68 @@ quantize_bf16_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint32_t* 
     }
 }
 
+// Same conversion, fed by plain 128-bit loads instead of the bulk-copy ring: warp u
+// of the grid converts 32-block units u, u + n_warps, ... (2 KB of bf16 each, read
+// as four fully coalesced 512-byte warp loads, non-allocating in L1), two units per
+// iteration so that 8 loads per lane are in flight.  Lane and block mapping and the
+// stores are those of quantize_bf16_kernel.
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void quant_unit_bf16(const uint4 (&v)[4], int64_t blk0, int64_t n_blocks, int lane,
+                                                uint32_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                int rule) {
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t am = amax8_bf16(v[j]);
+        am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+        am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+        const bool nf = am >= 0x7F80u;
+        const int s = block_exp_bf16(am, rule);
+        const uint32_t cw = nf ? 0u : quant8_bf16(v[j], inv_pow2(s));
+        const uint32_t S = nf ? 0xFFu : static_cast<uint32_t>(s + 127);
+        const int64_t blk = blk0 + 8 * j + (lane >> 2);
+        if (blk < n_blocks) __stcs(codes + blk0 * 4 + 32 * j + lane, cw);
+        const uint32_t got = __shfl_sync(0xFFFFFFFFu, S, (lane & 7) * 4);
+        if ((lane >> 3) == j) mine = got;
+    }
+    if (blk0 + lane < n_blocks) scales[blk0 + lane] = static_cast<uint8_t>(mine);
+}
+
+constexpr int kLsuThreads = 256;
+
+__global__ void __launch_bounds__(kLsuThreads)
+quantize_bf16_lsu_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint32_t* __restrict__ codes,
+                         uint8_t* __restrict__ scales, int rule) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * kLsuThreads + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * kLsuThreads) >> 5;
+    const int64_t n_units = (n_blocks + 31) / 32;
+    const int64_t n_vec = n_blocks * 4;   // 16-byte vectors of input
+    for (int64_t u = w0; u < n_units; u += 2 * nw) {
+        const int64_t u2 = u + nw;
+        uint4 a[4], b[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t i = u * 128 + 32 * j + lane;
+            a[j] = i < n_vec ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t i = u2 * 128 + 32 * j + lane;
+            b[j] = (u2 < n_units && i < n_vec) ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
+        }
+        quant_unit_bf16(a, u * 32, n_blocks, lane, codes, scales, rule);
+        if (u2 < n_units) quant_unit_bf16(b, u2 * 32, n_blocks, lane, codes, scales, rule);
+    }
+}
+
 // ---------------------------------------------------------------- fp32 -> MXFP4
 // Chunk = 256 blocks (32 KB of fp32).  Consumer warp w converts blocks
 // 32w .. 32w+31: step j (0..7) reads vectors 32j + l, i.e. block 4j + l/8, a
@@ -458,10 +520,13 @@ cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t col
             static_cast<const uint8_t*>(x), n_blocks, reinterpret_cast<uint16_t*>(codes), scales,
             rule, status);
     } else {
-        if ((e = set_ring_smem(quantize_bf16_kernel)) != cudaSuccess) return e;
-        quantize_bf16_kernel<<<grid, kRingThreads, kRingSmemBytes, stream>>>(
-            static_cast<const uint8_t*>(x), n_blocks, reinterpret_cast<uint32_t*>(codes), scales,
-            rule, status);
+        (void)status;
+        const int64_t n_units = (n_blocks + 31) / 32;
+        int64_t g = (n_units + 2 * (kLsuThreads / 32) - 1) / (2 * (kLsuThreads / 32));
+        const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+        if (g > cap) g = cap;
+        quantize_bf16_lsu_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), kLsuThreads, 0, stream>>>(
+            static_cast<const uint4*>(x), n_blocks, reinterpret_cast<uint32_t*>(codes), scales, rule);
     }
     return cudaGetLastError();
 }

@@ -19,7 +19,8 @@
 //                  per-chunk base ranks, and the expert's total;
 //   route_scatter  offsets (exclusive scan over experts, recomputed per CTA in
 //                  shared memory), the position of every pair, perm / inv /
-//                  sorted weights, and optionally the gather of token rows;
+//                  sorted weights / the token of every sorted row, and optionally
+//                  the gather of token rows (the W4A4 layer's packed rows);
 //   moe_combine    one thread per 8 output columns of a token:
 //                  out[t] = bf16(sum_j y[inv[t*k + j]]), fp32, slot order.
 #include "common.cuh"
@@ -186,7 +187,9 @@ route_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
     if (threadIdx.x == 0) counts[e] = total;
 }
 
-// One warp per pair: its sorted position, the routing tables and, if `x` is
+// One warp per pair: its sorted position, the routing tables (perm, inv, the
+// sorted routing weights and, if `row_tok` is given, the token of every sorted
+// row, which a GEMM that gathers its activation rows itself reads) and, if `x` is
 // given, the copy of its token's row into the expert-sorted activation matrix
 // (row_vec 16-byte vectors per row); if `xs` is given, likewise for a second
 // matrix of xs_row bytes per row (the block scales of MXFP4 activations).
@@ -197,7 +200,8 @@ route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
                      const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ local_rank,
                      const int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int64_t P,
                      int k, int E, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                     float* __restrict__ w_sorted, const uint4* __restrict__ x, int64_t row_vec,
+                     float* __restrict__ w_sorted, int32_t* __restrict__ row_tok,
+                     const uint4* __restrict__ x, int64_t row_vec,
                      uint4* __restrict__ x_sorted, const uint8_t* __restrict__ xs, int64_t xs_row,
                      uint8_t* __restrict__ xs_sorted) {
     __shared__ int32_t s_off[kMaxExperts];
@@ -225,6 +229,7 @@ route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
             perm[pos] = static_cast<int32_t>(p);
             inv[p] = static_cast<int32_t>(pos);
             if (w_sorted) w_sorted[pos] = weights[p];
+            if (row_tok) row_tok[pos] = static_cast<int32_t>(t);
         }
         if (x) {   // all of a lane's loads first, then its stores: 8 x 16 B in flight per lane
             const uint4* src = x + t * row_vec;
@@ -247,6 +252,41 @@ route_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ 
             const uint8_t* src = xs + t * xs_row;
             uint8_t* dst = xs_sorted + pos * xs_row;
             for (int64_t c = lane; c < xs_row; c += 32) dst[c] = __ldg(src + c);
+        }
+    }
+}
+
+// dst row i = src row idx[i] / div, for rows of row_vec vectors of type V (16-byte
+// or 4-byte); one warp per row, all of a lane's loads issued before its stores.  An
+// index outside the source leaves its row untouched and records
+// MXFP4_ERR_INVALID_ARG in the status word.
+template <typename V>
+__global__ void __launch_bounds__(kRouteThreads)
+gather_rows_kernel(const V* __restrict__ src, int64_t n_src, const int32_t* __restrict__ idx, int64_t n,
+                   int div, int64_t row_vec, V* __restrict__ dst, unsigned* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t i = warp0; i < n; i += nwarps) {
+        const int64_t r = __ldg(idx + i) / div;
+        if (r < 0 || r >= n_src) {
+            if (lane == 0) record_status(status, MXFP4_ERR_INVALID_ARG);
+            continue;
+        }
+        const V* s = src + r * row_vec;
+        V* d = dst + i * row_vec;
+        for (int64_t c0 = 0; c0 < row_vec; c0 += 32 * 8) {
+            V v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t c = c0 + lane + 32 * u;
+                if (c < row_vec) v[u] = __ldg(s + c);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t c = c0 + lane + 32 * u;
+                if (c < row_vec) d[c] = v[u];
+            }
         }
     }
 }
@@ -292,17 +332,39 @@ size_t route_tmp_bytes(int64_t T, int64_t E, int top_k) {
     return static_cast<size_t>(n_chunks * E + T * top_k) * sizeof(int32_t);
 }
 
+void route_tmp_split(void* tmp, int64_t T, int64_t E, int32_t** chunk_counts, int32_t** local_rank) {
+    const int64_t n_chunks = (T + kTokPerChunk - 1) / kTokPerChunk;
+    *chunk_counts = static_cast<int32_t*>(tmp);
+    *local_rank = *chunk_counts + n_chunks * E;
+}
+
 cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, int32_t* ids,
                          float* weights, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv, float* w_sorted, void* tmp, const void* x,
+                         int32_t* inv, float* w_sorted, int32_t* row_tok, void* tmp, const void* x,
                          int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
                          void* xs_sorted, int sm_count, cudaStream_t stream) {
     const int64_t n_chunks = (T + kTokPerChunk - 1) / kTokPerChunk;
-    int32_t* chunk_counts = static_cast<int32_t*>(tmp);
-    int32_t* local_rank = chunk_counts + n_chunks * E;
+    int32_t *chunk_counts, *local_rank;
+    route_tmp_split(tmp, T, E, &chunk_counts, &local_rank);
     route_topk_kernel<<<static_cast<unsigned>(n_chunks), kRouteThreads, 0, stream>>>(
         logits, static_cast<int>(T), static_cast<int>(E), top_k, ids, weights, chunk_counts,
         local_rank);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_route_finish(T, E, top_k, ids, weights, counts, offsets, perm, inv, w_sorted, row_tok,
+                               tmp, x, row_bytes, x_sorted, xs, xs_row_bytes, xs_sorted, sm_count, stream);
+}
+
+// The routing after top-k (chunk counts and ranks already in `tmp`): per-expert scan,
+// offsets, permutation tables and the optional row copies.
+cudaError_t launch_route_finish(int64_t T, int64_t E, int top_k, const int32_t* ids, const float* weights,
+                                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                                float* w_sorted, int32_t* row_tok, void* tmp, const void* x,
+                                int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
+                                void* xs_sorted, int sm_count, cudaStream_t stream) {
+    const int64_t n_chunks = (T + kTokPerChunk - 1) / kTokPerChunk;
+    int32_t *chunk_counts, *local_rank;
+    route_tmp_split(tmp, T, E, &chunk_counts, &local_rank);
     route_scan_kernel<<<static_cast<unsigned>(E), kRouteThreads, 0, stream>>>(
         chunk_counts, static_cast<int>(n_chunks), static_cast<int>(E), counts);
     const int64_t P = T * top_k;
@@ -311,9 +373,26 @@ cudaError_t launch_route(const float* logits, int64_t T, int64_t E, int top_k, i
     if (grid > cap) grid = cap;
     route_scatter_kernel<<<static_cast<unsigned>(grid), kRouteThreads, 0, stream>>>(
         ids, weights, chunk_counts, local_rank, counts, offsets, P, top_k, static_cast<int>(E),
-        perm, inv, w_sorted, static_cast<const uint4*>(x), row_bytes / 16,
+        perm, inv, w_sorted, row_tok, static_cast<const uint4*>(x), row_bytes / 16,
         static_cast<uint4*>(x_sorted), static_cast<const uint8_t*>(xs), xs_row_bytes,
         static_cast<uint8_t*>(xs_sorted));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* src, int64_t n_src, int64_t row_bytes, const int32_t* idx,
+                               int64_t n, int div, void* dst, int sm_count, unsigned* status,
+                               cudaStream_t stream) {
+    int64_t grid = (n + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
+    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    if (row_bytes % 16 == 0)
+        gather_rows_kernel<uint4><<<static_cast<unsigned>(grid), kRouteThreads, 0, stream>>>(
+            static_cast<const uint4*>(src), n_src, idx, n, div, row_bytes / 16, static_cast<uint4*>(dst), status);
+    else
+        gather_rows_kernel<uint32_t><<<static_cast<unsigned>(grid), kRouteThreads, 0, stream>>>(
+            static_cast<const uint32_t*>(src), n_src, idx, n, div, row_bytes / 4, static_cast<uint32_t*>(dst),
+            status);
     return cudaGetLastError();
 }
 

@@ -52,16 +52,6 @@ constexpr int kRateA = 0, kRateB = 16384, kRateBar = 16384 + 32768;
 constexpr int kRateSmem = 116 * 1024;
 static_assert(kRateBar + 64 + 1024 <= kRateSmem, "probe layout");
 
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __global__ void __launch_bounds__(kRateThreads, 1)
 selftest_mma_rate_kernel(int kind, int iters, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];

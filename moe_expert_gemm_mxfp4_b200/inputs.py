@@ -16,6 +16,9 @@ hidden H = 2880, expert intermediate I = 2880, top-4 routing):
                     the router logits (load imbalance).
 * ``moe_120b``    – T=4096 tokens, 128 experts, top-4.
 
+The router-projection recipe draws bf16 router weights W_r [E, H] ~ N(0, 1/H)
+(sub-seed of the layer's seed), so that x . W_r^T ~ N(0, 1) like the logits.
+
 For the MoE recipes x ~ N(0,1) (bf16), router logits ~ N(0,1) (fp32) and each
 expert's gate_up weight [2I, H] (rows [0, I) gate, [I, 2I) up) and down weight
 [H, I] ~ N(0, 0.02) (fp32), drawn expert by expert from sub-seeds so that any
@@ -29,7 +32,7 @@ import torch
 
 __all__ = [
     "MoEConfig", "MOE_CONFIGS", "gemm_small", "quant_tensor", "moe_activations",
-    "expert_weights", "seeded_bf16", "seeded_f32",
+    "expert_weights", "seeded_bf16", "seeded_f32", "router_weights",
 ]
 
 
@@ -128,3 +131,8 @@ def expert_weights(cfg: MoEConfig, e: int):
     w13 = seeded_f32((2 * cfg.I, cfg.H), expert_seed(cfg.seed, e, 0), cfg.w_std)
     w2 = seeded_f32((cfg.H, cfg.I), expert_seed(cfg.seed, e, 1), cfg.w_std)
     return w13, w2
+
+
+def router_weights(cfg: "MoEConfig") -> torch.Tensor:
+    """bf16 router weights [E, H] ~ N(0, 1/H) (std 1/sqrt(H)) from a sub-seed of cfg.seed."""
+    return seeded_bf16((cfg.E, cfg.H), cfg.seed * 1_000_003 + 999_983, cfg.H ** -0.5)

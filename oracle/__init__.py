@@ -40,7 +40,7 @@ from . import build as _build
 __all__ = [
     "E2M1_GRID", "FLOOR", "CEIL", "e2m1_magnitude", "bf16_to_f64", "f64_to_bf16",
     "quantize", "dequantize_bf16", "dequantize_f64", "route", "gemm_w4a16",
-    "gemm_w4a4", "moe_mlp", "silu",
+    "gemm_w4a4", "moe_mlp", "moe_down", "silu", "router_logits",
 ]
 
 FLOOR = 0
@@ -163,6 +163,21 @@ def dequantize_bf16(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 # --------------------------------------------------------------------------- routing
 
+def router_logits(x_bits: np.ndarray, w_router_bits: np.ndarray) -> np.ndarray:
+    """Router projection: logits[t, e] = sum_h x[t, h] * W_r[e, h] with bf16 x [T, H]
+    and bf16 router weights W_r [E, H], in fp64 (returned unrounded).
+
+    Reading: the pages route each token through the MoE kernel's top-k ([P4]
+    "Zero-Build Kernels from the Hub", MegaBlocks MoE) without printing the router;
+    the plainest router is a bias-free linear map of the token to one logit per
+    expert, its operands in the layer's bf16.
+    """
+    x = bf16_to_f64(_as_bf16_bits(x_bits))
+    w = bf16_to_f64(_as_bf16_bits(w_router_bits))
+    return x @ w.T
+
+
+
 def route(logits: np.ndarray, top_k: int):
     """Top-k routing, softmax over the k selected logits, and the expert-sorted
     permutation of the (token, slot) pairs.
@@ -284,4 +299,32 @@ def moe_mlp(x_bits, logits, top_k, w13_codes, w13_scales, w2_codes, w2_scales,
         np.add.at(out, rows, w[rows, slots][:, None] * y)
     if return_h:
         return out, h_all
+    return out
+
+
+def moe_down(h_bits, logits, top_k, w2_codes, w2_scales, mode: str = "w4a16", tokens=None):
+    """The second half of ``moe_mlp`` from a given h: for each token t and slot j
+    with expert e (``route``),
+        y = h_tj . W2[e]^T          (``mode='w4a4'``: h_tj MXFP4-quantized first)
+    and out_t = sum_j w_tj * y_j in fp64 (returned unrounded).
+
+    h_bits: bf16 bit patterns [n_tokens, top_k, I] of the h rows of ``tokens`` (all
+    tokens if None), slot-major per token like ``moe_mlp(..., return_h=True)``.
+    This is the staged check's reference: fed with another implementation's h, it
+    isolates that implementation's down projection and combine from the rounding
+    of h (in W4A4 a last-bit difference in h can flip one of its MXFP4 codes).
+    """
+    h_bits = _as_bf16_bits(h_bits)
+    r = route(logits, top_k)
+    T = r["ids"].shape[0]
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    n, H = tok.size, w2_codes.shape[1]
+    ids, w = r["ids"][tok], r["w"][tok]
+    out = np.zeros((n, H), dtype=np.float64)
+    for e in np.unique(ids):
+        rows, slots = np.nonzero(ids == e)
+        hb = h_bits[rows, slots]
+        h = _fake_quant_bf16(hb) if mode == "w4a4" else bf16_to_f64(hb)
+        y = h @ _deq_weights(w2_codes[e], w2_scales[e]).T
+        np.add.at(out, rows, w[rows, slots][:, None] * y)
     return out

@@ -90,3 +90,15 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_LIB", None)
     with pytest.raises(_lib.Mxfp4LibraryMissing):
         _lib.load(str(tmp_path / "nope.so"))
+
+
+def test_workspace_layout_mirror_matches_the_library():
+    # the tests' copy of the workspace carving (used to read h for the W4A4 staged
+    # check) must describe the library's workspace exactly
+    from helpers import moe_ws_layout
+    lib = _lib.load()
+    for T, H, I, E, k in ((1, 64, 64, 1, 1), (37, 192, 128, 8, 2), (256, 2880, 2880, 32, 4),
+                          (4096, 2880, 2880, 128, 4), (513, 64, 128, 3, 1)):
+        for mode in (0, 1):
+            assert moe_ws_layout(T, H, I, E, k, mode == 1)["total"] == \
+                lib.moe_mxfp4_workspace_size(T, H, I, E, k, mode), (T, H, I, E, k, mode)

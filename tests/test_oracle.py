@@ -360,6 +360,46 @@ def test_route_nan_logits_rank_below_every_number():
     assert np.all(np.isfinite(r["w"][4:]))
 
 
+def test_moe_down_fed_with_moe_mlp_h_reproduces_moe_mlp():
+    # the staged check's reference: moe_down(h of moe_mlp) is moe_mlp, bit for bit,
+    # in both modes
+    g = torch.Generator().manual_seed(23)
+    T, H, I, E, k = 9, 64, 96, 5, 2
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    logits = torch.randn(T, E, generator=g).numpy()
+    q13 = [oracle.quantize((torch.randn(2 * I, H, generator=g) * 0.1).numpy()) for _ in range(E)]
+    q2 = [oracle.quantize((torch.randn(H, I, generator=g) * 0.1).numpy()) for _ in range(E)]
+    w13c, w13s = np.stack([a for a, _ in q13]), np.stack([b for _, b in q13])
+    w2c, w2s = np.stack([a for a, _ in q2]), np.stack([b for _, b in q2])
+    for mode in ("w4a16", "w4a4"):
+        out, h = oracle.moe_mlp(xb, logits, k, w13c, w13s, w2c, w2s, mode=mode, return_h=True)
+        hb = oracle.f64_to_bf16(h)
+        assert np.array_equal(oracle.moe_down(hb, logits, k, w2c, w2s, mode=mode), out)
+        tok = np.array([1, 4, 8])
+        assert np.array_equal(oracle.moe_down(hb[tok], logits, k, w2c, w2s, mode=mode, tokens=tok), out[tok])
+
+
+def test_router_logits_bruteforce():
+    g = torch.Generator().manual_seed(24)
+    T, E, H = 5, 7, 96
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    w = (torch.randn(E, H, generator=g) * 0.1).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    got = oracle.router_logits(xb, wb)
+    assert got.shape == (T, E)
+    xf, wf = x.double().numpy(), w.double().numpy()
+    for t in range(T):
+        for e in range(E):
+            assert got[t, e] == pytest.approx(math.fsum(float(xf[t, h]) * float(wf[e, h]) for h in range(H)),
+                                              rel=1e-15, abs=1e-300)
+    # a one-hot token picks a router column exactly; transposed operands would not
+    onehot = np.zeros((1, H), np.uint16)
+    onehot[0, 17] = 0x3F80                     # 1.0
+    assert np.array_equal(oracle.router_logits(onehot, wb)[0], wf[:, 17])
+
+
 # ----------------------------------------------------------------- GEMM
 
 def test_gemm_bruteforce():
