@@ -448,6 +448,38 @@ def bench_route_project(dev, steps=20, warmup=5):
     return out
 
 
+def bench_bf16_line(name, cfg, dev, pk, mxfp4_line=None, steps=10, warmup=3):
+    """The same layer with bf16 expert weights (moe_bf16_mlp, the comparison the pages
+    draw against MXFP4): per-layer time, weight GB/s and the MXFP4 layer's speed-up."""
+    import moe_expert_gemm_mxfp4_b200 as mx
+    from moe_expert_gemm_mxfp4_b200 import inputs
+    E, H, I = cfg.E, cfg.H, cfg.I
+    w13 = torch.empty((E, 2 * I, H), dtype=torch.bfloat16, device=dev)
+    w2 = torch.empty((E, H, I), dtype=torch.bfloat16, device=dev)
+    for e in range(E):
+        a, b = inputs.expert_weights(cfg, e)
+        w13[e].copy_(a.to(dev))
+        w2[e].copy_(b.to(dev))
+    x, logits = inputs.moe_activations(cfg)
+    x, logits = x.to(dev), logits.to(dev)
+    out = torch.empty((cfg.T, H), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((mx.moe_bf16_workspace_size(cfg.T, H, I, E, cfg.top_k),), dtype=torch.uint8, device=dev)
+    ms = time_kernel(lambda i: mx.moe_bf16_mlp(x, logits, cfg.top_k, w13, w2, out=out, ws=ws), steps, warmup, dev)
+    assert mx.mxfp4_get_device_status() == 0
+    n_act = torch.topk(logits, cfg.top_k, dim=1).indices.unique().numel()
+    wbytes = n_act * (2 * I * H + H * I) * 2
+    fl = layer_flops(cfg.T, cfg.top_k, H, I)
+    line = {"workload": f"{name}: T={cfg.T} E={E} top-{cfg.top_k} H={H} I={I} bf16 weights",
+            "us_per_layer": ms * 1e3, "tflops": fl / ms / 1e9, "weight_gbs": wbytes / ms / 1e6,
+            "frac_hbm_weights": wbytes / ms / 1e6 / pk["hbm"], "frac_bf16": fl / ms / 1e9 / pk["bf16"],
+            "weight_bytes": wbytes}
+    if mxfp4_line:
+        line["mxfp4_speedup"] = ms * 1e3 / mxfp4_line["us_per_layer"]
+    del w13, w2
+    torch.cuda.empty_cache()
+    return line
+
+
 def breakdown(dev, pk):
     import moe_expert_gemm_mxfp4_b200 as mx
     from moe_expert_gemm_mxfp4_b200 import inputs
@@ -459,6 +491,7 @@ def breakdown(dev, pk):
     L = gpu_layer(cfg, dev)
     bd["moe_decode"] = bench_moe_line("moe_decode", cfg, L, mx.W4A16, dev, pk, steps=20)
     del L
+    bd["moe_decode_bf16_weights"] = bench_bf16_line("moe_decode", cfg, dev, pk, bd["moe_decode"])
     cfg = inputs.MOE_CONFIGS["moe_120b"]
     L = gpu_layer(cfg, dev)
     bd["moe_120b_w4a16"] = bench_moe_line("moe_120b", cfg, L, mx.W4A16, dev, pk)
@@ -588,9 +621,18 @@ def run_profile_case(args):
         for _ in range(n):
             c, sc = mx.mxfp4_quantize(x)
             mx.mxfp4_dequantize(c, sc)
+    elif args.profile in ("route_project_decode", "route_project_prefill"):
+        cfg = inputs.MOE_CONFIGS["moe_decode" if args.profile.endswith("decode") else "moe_prefill"]
+        x, _ = inputs.moe_activations(cfg)
+        x, w = x.to(dev), inputs.router_weights(cfg).to(dev)
+        for _ in range(n):
+            mx.moe_mxfp4_route_project(x, w, cfg.top_k)
     else:
-        cfg = inputs.MOE_CONFIGS["moe_decode" if args.profile == "decode" else "moe_120b"]
-        mode = mx.W4A16 if args.profile == "decode" else mx.W4A4
+        cfg = inputs.MOE_CONFIGS[{"decode": "moe_decode", "prefill": "moe_prefill"}.get(args.profile, "moe_120b")]
+        if args.tokens:
+            import dataclasses
+            cfg = dataclasses.replace(cfg, T=args.tokens)
+        mode = mx.W4A4 if args.profile == "w4a4_120b" else mx.W4A16
         L = gpu_layer(cfg, dev)
         xd, ld = L["x"].to(dev), L["logits"].to(dev)
         out = torch.empty((xd.shape[0], cfg.H), dtype=torch.bfloat16, device=dev)
@@ -617,7 +659,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the prefill workload (profiling runs on a smaller case)")
-    ap.add_argument("--profile", choices=["decode", "w4a4_120b", "quant"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "w4a4_120b", "quant", "route_project_decode",
+                                          "route_project_prefill"], default=None,
                     help="run one breakdown workload --warmup + --steps times, untimed, and "
                          "print a status line (a driver for ncu captures)")
     args = ap.parse_args()
@@ -689,6 +732,8 @@ def main():
     torch.cuda.empty_cache()
     if not args.no_breakdown and world == 1:
         line["breakdown"] = breakdown(dev, pk)
+        line["breakdown"]["moe_prefill_bf16_weights"] = bench_bf16_line(
+            "moe_prefill", cfg, dev, pk, {"us_per_layer": step_ms * 1e3})
     if not args.no_cpu and world == 1:
         line["cpu_baseline"] = cpu_baseline(cfg)
     print(json.dumps(line), flush=True)

@@ -217,6 +217,22 @@ MXFP4_API size_t moe_mxfp4_experts_workspace_size(int64_t P, int64_t H, int64_t 
 MXFP4_API mxfp4_status moe_mxfp4_combine(const float* y_sorted, const int32_t* inv, int64_t T,
                                          int32_t top_k, int64_t H, void* out_bf16, void* stream);
 
+/* ---------------------------------------------------------------- bf16-weight layer (comparison)
+ * The same layer as moe_mxfp4_mlp in W4A16 arithmetic, with the expert weights in bf16
+ * instead of MXFP4: w13 bf16 [E, 2I, H] (rows [0, I) gate, [I, 2I) up), w2 bf16
+ * [E, H, I]; everything else (routing, SwiGLU, fp32 accumulation, weighted combine,
+ * x, logits, out, ws = moe_bf16_workspace_size() bytes) as moe_mxfp4_mlp.  It exists to
+ * measure what MXFP4 weights save on this GPU against the format they replace.
+ * Requires H % 64 == 0 and I % 64 == 0.
+ * Source: agentlenshq.com, "Transformers 4.40 performance upgrades for OpenAI
+ * GPT-OSS ...", sections "Native Support in transformers" (without the MXFP4 path the
+ * model runs in bfloat16 at roughly four times the memory) and "Memory Savings". */
+MXFP4_API mxfp4_status moe_bf16_mlp(const void* x_bf16, int64_t T, int64_t H, const float* router_logits,
+                                    int64_t E, int32_t top_k, const void* w13_bf16, int64_t I,
+                                    const void* w2_bf16, void* out_bf16, void* ws, size_t ws_bytes,
+                                    void* stream);
+MXFP4_API size_t moe_bf16_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k);
+
 /* ---------------------------------------------------------------- allocation-free MoE layer
  * Not a step of the method: the pages have no counterpart of this entry point.
  *

@@ -27,7 +27,7 @@ __all__ = [
     "moe_mxfp4_workspace_size", "moe_mxfp4_mlp_noalloc", "mxfp4_get_device_status",
     "mxfp4_selftest_wait_timeout", "mxfp4_selftest_mma_rate", "mxfp4_set_trace_events",
     "moe_mxfp4_route_project", "mxfp4_gather_rows", "moe_mxfp4_experts",
-    "moe_mxfp4_experts_workspace_size", "moe_mxfp4_combine",
+    "moe_mxfp4_experts_workspace_size", "moe_mxfp4_combine", "moe_bf16_mlp", "moe_bf16_workspace_size",
     "Mxfp4Error", "Mxfp4LibraryMissing",
     "SCALE_FLOOR", "SCALE_CEIL", "W4A16", "W4A4", "library_path",
 ]
@@ -289,6 +289,40 @@ def moe_mxfp4_combine(y_sorted: torch.Tensor, inv: torch.Tensor, top_k: int, out
     _on_current_device(y_sorted=y_sorted, inv=inv, out=out)
     _lib.check("moe_mxfp4_combine", _lib.load().moe_mxfp4_combine(
         _p(y_sorted), _p(inv), T, top_k, H, _p(out), _stream(stream)))
+    return out
+
+
+def moe_bf16_workspace_size(T, H, I, E, top_k) -> int:
+    return int(_lib.load().moe_bf16_workspace_size(T, H, I, E, top_k))
+
+
+def moe_bf16_mlp(x: torch.Tensor, logits: torch.Tensor, top_k: int, w13: torch.Tensor, w2: torch.Tensor,
+                 out=None, ws=None, stream=None):
+    """The MoE layer with bf16 expert weights (the comparison for moe_mxfp4_mlp):
+    w13 bf16 [E, 2I, H], w2 bf16 [E, H, I]."""
+    _need_dims(x, "x", 2)
+    _need_dims(logits, "logits", 2)
+    _need_dims(w13, "w13", 3)
+    T, H = x.shape
+    E, twoI, _ = w13.shape
+    I = twoI // 2
+    _need(x, "x", torch.bfloat16)
+    _need(logits, "logits", torch.float32, (T, E))
+    _need(w13, "w13", torch.bfloat16, (E, 2 * I, H))
+    _need(w2, "w2", torch.bfloat16, (E, H, I))
+    if out is None:
+        out = _empty((T, H), torch.bfloat16, x)
+    else:
+        _need(out, "out", torch.bfloat16, (T, H))
+    need = moe_bf16_workspace_size(T, H, I, E, top_k)
+    if ws is None:
+        ws = _empty((need,), torch.uint8, x)
+    else:
+        _need(ws, "ws")
+    _on_current_device(x=x, logits=logits, w13=w13, w2=w2, out=out, ws=ws)
+    _lib.check("moe_bf16_mlp", _lib.load().moe_bf16_mlp(
+        _p(x), T, H, _p(logits), E, top_k, _p(w13), I, _p(w2), _p(out), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
     return out
 
 

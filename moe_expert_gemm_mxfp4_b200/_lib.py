@@ -65,6 +65,8 @@ _SIGS = {
                                          ctypes.c_int, _vp, _sz, _vp]),
     "moe_mxfp4_experts_workspace_size": (_sz, [_i64, _i64, _i64, _i64, ctypes.c_int]),
     "moe_mxfp4_combine": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i64, _vp, _vp]),
+    "moe_bf16_mlp": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "moe_bf16_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32]),
     "mxfp4_get_device_status": (ctypes.c_int, [_vp]),
     "mxfp4_selftest_wait_timeout": (ctypes.c_int, [_vp]),
     "mxfp4_selftest_mma_rate": (ctypes.c_int, [_i32, _i32, ctypes.POINTER(ctypes.c_double), _vp]),

@@ -137,6 +137,22 @@ mxfp4_status encode_x4_map(CUtensorMap* m, const uint8_t* codes, int64_t K, int6
     return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
 }
 
+// bf16 weights of G groups as a 3-D tensor {K, rows, G}; box {64, box_rows, 1}
+// (128 B of K per row per copy); 128-byte swizzle (UMMA K-major SW128 layout).
+mxfp4_status encode_w16_map(CUtensorMap* m, const void* w, int64_t K, int64_t rows, int64_t G, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(G)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K * 2), static_cast<cuuint64_t>(rows * K * 2)};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MXFP4_OK : cuda_fail(cudaErrorInvalidValue);
+}
+
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace of moe_mxfp4_mlp, carved in this order (256-byte aligned pieces).
@@ -231,11 +247,7 @@ mxfp4_status run_experts(DeviceInfo* d, int64_t P, int64_t H, int64_t I, int64_t
     const bool a4 = mode == MXFP4_W4A4;
     mxfp4_status st;
     cudaError_t e;
-    // W4A16 with at most 32 rows per expert on average: the small-group (mma.sync) engine
-    const int nt_h = a4 ? 0 : mx::pick_token_tiling_hmma(P, E);
-    const bool small = nt_h > 0 && mx::hmma_fits_k(H) && mx::hmma_fits_k(I);
-    mx::TokenTiling tiling = a4 ? mx::pick_token_tiling_w4a4(P, E) : mx::pick_token_tiling(P, E);
-    if (small) tiling = {nt_h, 1};
+    const mx::TokenTiling tiling = a4 ? mx::pick_token_tiling_w4a4(P, E) : mx::pick_token_tiling(P, E);
     const int64_t tile_rows = static_cast<int64_t>(tiling.nt) * tiling.tt;
     const int64_t tok_tiles = (P + tile_rows - 1) / tile_rows + E;
 
@@ -262,7 +274,6 @@ mxfp4_status run_experts(DeviceInfo* d, int64_t P, int64_t H, int64_t I, int64_t
     a.status = d->status;
     const int grid1 = gemm_grid(d, tok_tiles * a.n_ftiles);
     e = a4      ? mx::launch_grouped_gemm_w4a4(mx::EPI_SWIGLU, tiling.nt, tw, tx, a, grid1, s)
-        : small ? mx::launch_grouped_gemm_hmma(mx::EPI_SWIGLU, tiling.nt, tw, tx, a, grid1, s)
                 : mx::launch_grouped_gemm(mx::EPI_SWIGLU, tiling, tw, tx, a, grid1, s);
     if (e != cudaSuccess) return cuda_fail(e);
 
@@ -289,7 +300,6 @@ mxfp4_status run_experts(DeviceInfo* d, int64_t P, int64_t H, int64_t I, int64_t
     a.row_w = io.row_w;
     const int grid2 = gemm_grid(d, tok_tiles * a.n_ftiles);
     e = a4      ? mx::launch_grouped_gemm_w4a4(mx::EPI_WEIGHTED, tiling.nt, tw, tx, a, grid2, s)
-        : small ? mx::launch_grouped_gemm_hmma(mx::EPI_WEIGHTED, tiling.nt, tw, tx, a, grid2, s)
                 : mx::launch_grouped_gemm(mx::EPI_WEIGHTED, tiling, tw, tx, a, grid2, s);
     if (e != cudaSuccess) return cuda_fail(e);
     trace_mark(3, s);
@@ -447,11 +457,8 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     mxfp4_status st = device_info(&d);
     if (st != MXFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    mx::TokenTiling tiling =
+    const mx::TokenTiling tiling =
         mode == MXFP4_W4A4 ? mx::pick_token_tiling_w4a4(M, 1) : mx::pick_token_tiling(M, 1);
-    const int nt_h = mode == MXFP4_W4A4 ? 0 : mx::pick_token_tiling_hmma(M, 1);
-    const bool small = nt_h > 0 && mx::hmma_fits_k(K);   // at most 32 rows: the mma.sync engine
-    if (small) tiling = {nt_h, 1};
     CUtensorMap tw, tx;
     if ((st = encode_codes_map(&tw, w_codes, K, N, 1, 128)) != MXFP4_OK) return st;
     uint8_t* xq_codes = static_cast<uint8_t*>(ws);
@@ -485,7 +492,6 @@ mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t*
     cudaError_t e = mode == MXFP4_W4A4
                         ? mx::launch_grouped_gemm_w4a4(mx::EPI_PLAIN, tiling.nt, tw, tx, a,
                                                        gemm_grid(d, tiles), s)
-                    : small ? mx::launch_grouped_gemm_hmma(mx::EPI_PLAIN, tiling.nt, tw, tx, a, gemm_grid(d, tiles), s)
                             : mx::launch_grouped_gemm(mx::EPI_PLAIN, tiling, tw, tx, a,
                                                       gemm_grid(d, tiles), s);
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
@@ -716,6 +722,78 @@ mxfp4_status moe_mxfp4_combine(const float* y_sorted, const int32_t* inv, int64_
     cudaError_t e = mx::launch_combine(y_sorted, inv, T, top_k, H, out_bf16, d->sm_count,
                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXFP4_OK : cuda_fail(e);
+}
+
+mxfp4_status moe_bf16_mlp(const void* x_bf16, int64_t T, int64_t H, const float* router_logits, int64_t E,
+                          int32_t top_k, const void* w13_bf16, int64_t I, const void* w2_bf16, void* out_bf16,
+                          void* ws, size_t ws_bytes, void* stream) {
+    mxfp4_status st = check_route_args(router_logits, T, E, top_k);
+    if (st != MXFP4_OK) return st;
+    if (!x_bf16 || !w13_bf16 || !w2_bf16 || !out_bf16) return MXFP4_ERR_INVALID_ARG;
+    if (H <= 0 || I <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (H % 64 != 0 || I % 64 != 0 || H >= (int64_t{1} << 31) || I >= (int64_t{1} << 31))
+        return MXFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(router_logits) || !aligned16(w13_bf16) || !aligned16(w2_bf16) ||
+        !aligned16(out_bf16))
+        return MXFP4_ERR_MISALIGNED;
+    const size_t need = moe_bf16_workspace_size(T, H, I, E, top_k);
+    if (!ws || ws_bytes < need) return MXFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MXFP4_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((st = device_info(&d)) != MXFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const MoeWs w = carve_moe(ws, T, H, I, E, top_k, MXFP4_W4A16);
+    const int64_t P = T * top_k;
+    trace_mark(0, s);
+    cudaError_t e = mx::launch_route(router_logits, T, E, top_k, w.ids, w.weights, w.counts, w.offsets, w.perm,
+                                     w.inv, w.w_sorted, nullptr, w.route_tmp, x_bf16, H * 2, w.x_sorted, nullptr,
+                                     0, nullptr, d->sm_count, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    trace_mark(1, s);
+    const int nt = mx::pick_token_tiling_bf16w(P, E);
+    const int64_t tok_tiles = (P + nt - 1) / nt + E;
+    // gate/up with the SwiGLU epilogue: the weight tile in 16-row boxes (gate, up interleaved)
+    CUtensorMap tw, tx;
+    if ((st = encode_w16_map(&tw, w13_bf16, H, 2 * I, E, 16)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, w.x_sorted, H, P, nt)) != MXFP4_OK) return st;
+    mx::GemmArgs a{};
+    a.offsets = w.offsets;
+    a.G = static_cast<int>(E);
+    a.K = static_cast<int>(H);
+    a.rows_w = static_cast<int>(2 * I);
+    a.I = static_cast<int>(I);
+    a.n_ftiles = static_cast<int>(I / 64);
+    a.out = w.h;
+    a.out_ld = I;
+    a.n_valid_feat = static_cast<int>(I);
+    a.status = d->status;
+    if ((e = mx::launch_grouped_gemm_bf16w(mx::EPI_SWIGLU, nt, tw, tx, a, gemm_grid(d, tok_tiles * a.n_ftiles), s)) !=
+        cudaSuccess)
+        return cuda_fail(e);
+    trace_mark(2, s);
+    // down projection, routing weight applied in fp32
+    if ((st = encode_w16_map(&tw, w2_bf16, I, H, E, 128)) != MXFP4_OK) return st;
+    if ((st = encode_act_map(&tx, w.h, I, P, nt)) != MXFP4_OK) return st;
+    a.K = static_cast<int>(I);
+    a.rows_w = static_cast<int>(H);
+    a.I = 0;
+    a.n_ftiles = static_cast<int>((H + 127) / 128);
+    a.out = w.y_sorted;
+    a.out_ld = H;
+    a.n_valid_feat = static_cast<int>(H);
+    a.row_w = w.w_sorted;
+    if ((e = mx::launch_grouped_gemm_bf16w(mx::EPI_WEIGHTED, nt, tw, tx, a, gemm_grid(d, tok_tiles * a.n_ftiles), s)) !=
+        cudaSuccess)
+        return cuda_fail(e);
+    trace_mark(3, s);
+    if ((e = mx::launch_combine(w.y_sorted, w.inv, T, top_k, H, out_bf16, d->sm_count, s)) != cudaSuccess)
+        return cuda_fail(e);
+    trace_mark(4, s);
+    return MXFP4_OK;
+}
+
+size_t moe_bf16_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int32_t top_k) {
+    return moe_mxfp4_workspace_size(T, H, I, E, top_k, MXFP4_W4A16);
 }
 
 // ---------------------------------------------------------------- allocation-free MoE layer

@@ -71,13 +71,13 @@ cudaError_t launch_combine(const void* y_sorted, const int32_t* inv, int64_t T, 
                            int64_t H, void* out, int sm_count, cudaStream_t stream);
 TokenTiling pick_token_tiling(int64_t rows, int64_t groups);
 int64_t max_gemm_k();   // largest contraction length the grouped GEMM accepts
+
 cudaError_t launch_grouped_gemm(int mode, TokenTiling tiling, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_x, const GemmArgs& args, int grid,
                                 cudaStream_t stream);
-int pick_token_tiling_hmma(int64_t rows, int64_t groups);   // 16, 32, or 0 (groups too large)
-bool hmma_fits_k(int64_t K);
-cudaError_t launch_grouped_gemm_hmma(int mode, int nt, const CUtensorMap& tmap_w, const CUtensorMap& tmap_x,
-                                     const GemmArgs& args, int grid, cudaStream_t stream);
+int pick_token_tiling_bf16w(int64_t rows, int64_t groups);   // 64, 128 or 256
+cudaError_t launch_grouped_gemm_bf16w(int mode, int nt, const CUtensorMap& tmap_w, const CUtensorMap& tmap_x,
+                                      const GemmArgs& args, int grid, cudaStream_t stream);
 int64_t max_gemm_k_w4a4();   // largest contraction length the W4A4 engine accepts
 TokenTiling pick_token_tiling_w4a4(int64_t rows, int64_t groups);
 cudaError_t launch_grouped_gemm_w4a4(int mode, int nt, const CUtensorMap& tmap_w,

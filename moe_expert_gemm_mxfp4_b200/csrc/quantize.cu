@@ -319,30 +319,32 @@ __device__ __forceinline__ void quant_unit_bf16(const uint4 (&v)[4], int64_t blk
 }
 
 constexpr int kLsuThreads = 256;
+constexpr int kLsuUnits = 4;   // 32-block units in flight per warp (16 loads per lane)
 
+// Warp w of the grid converts the contiguous range of units [w * n / W, (w + 1) * n / W)
+// (W warps, n units: every warp gets the same count to within one), kLsuUnits at a
+// time with all their loads issued before any conversion.
 __global__ void __launch_bounds__(kLsuThreads)
 quantize_bf16_lsu_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint32_t* __restrict__ codes,
                          uint8_t* __restrict__ scales, int rule) {
     const int lane = threadIdx.x & 31;
-    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * kLsuThreads + threadIdx.x) >> 5;
+    const int64_t w = (static_cast<int64_t>(blockIdx.x) * kLsuThreads + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * kLsuThreads) >> 5;
     const int64_t n_units = (n_blocks + 31) / 32;
+    const int64_t u_end = (w + 1) * n_units / nw;
     const int64_t n_vec = n_blocks * 4;   // 16-byte vectors of input
-    for (int64_t u = w0; u < n_units; u += 2 * nw) {
-        const int64_t u2 = u + nw;
-        uint4 a[4], b[4];
+    for (int64_t u = w * n_units / nw; u < u_end; u += kLsuUnits) {
+        uint4 v[kLsuUnits][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t i = u * 128 + 32 * j + lane;
-            a[j] = i < n_vec ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
-        }
+        for (int k = 0; k < kLsuUnits; ++k)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t i = u2 * 128 + 32 * j + lane;
-            b[j] = (u2 < n_units && i < n_vec) ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
-        }
-        quant_unit_bf16(a, u * 32, n_blocks, lane, codes, scales, rule);
-        if (u2 < n_units) quant_unit_bf16(b, u2 * 32, n_blocks, lane, codes, scales, rule);
+            for (int j = 0; j < 4; ++j) {
+                const int64_t i = (u + k) * 128 + 32 * j + lane;
+                v[k][j] = (u + k < u_end && i < n_vec) ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+        for (int k = 0; k < kLsuUnits; ++k)
+            if (u + k < u_end) quant_unit_bf16(v[k], (u + k) * 32, n_blocks, lane, codes, scales, rule);
     }
 }
 
@@ -522,8 +524,14 @@ cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t col
     } else {
         (void)status;
         const int64_t n_units = (n_blocks + 31) / 32;
-        int64_t g = (n_units + 2 * (kLsuThreads / 32) - 1) / (2 * (kLsuThreads / 32));
-        const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+        // one wave of resident CTAs (each warp then owns an equal contiguous range), fewer
+        // when there are not kLsuUnits units per warp
+        int per_sm = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_bf16_lsu_kernel, kLsuThreads, 0)) !=
+            cudaSuccess)
+            return e;
+        int64_t g = (n_units + kLsuUnits * (kLsuThreads / 32) - 1) / (kLsuUnits * (kLsuThreads / 32));
+        const int64_t cap = static_cast<int64_t>(sm_count) * (per_sm > 0 ? per_sm : 1);
         if (g > cap) g = cap;
         quantize_bf16_lsu_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), kLsuThreads, 0, stream>>>(
             static_cast<const uint4*>(x), n_blocks, reinterpret_cast<uint32_t*>(codes), scales, rule);

@@ -20,7 +20,9 @@
 // Roles (one CTA per 128 tokens, 4 warps): thread 0 streams the x and W_r tiles of
 // each 64-wide K stage into a ring (TMA, 128B swizzle); thread 32 issues the MMAs
 // and releases each stage with a commit; afterwards all 128 threads run the top-k
-// epilogue.  Every wait is bounded (MXFP4_ERR_TIMEOUT in the status word).
+// epilogue.  Every wait is bounded (MXFP4_ERR_TIMEOUT in the status word); the
+// pipeline's waits poll without suspending the thread (one CTA's K loop is a chain of
+// such waits, so a late wake-up would cost each stage).
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,20 +33,24 @@ namespace {
 constexpr int kRpTok = 128;        // tokens per CTA = TMEM lanes
 constexpr int kRpThreads = 128;
 constexpr int kRpBK = 64;          // K per stage (128 bytes of bf16 per row)
-constexpr int kRpStages = 4;
+constexpr int kRpMaxStages = 12;   // ring depth: as many stages as fit (a K stage is a round trip to L2/HBM)
+constexpr int kRpSmemLimit = 227 * 1024;
 constexpr int kRpMaxTopK = 8;
 constexpr int kRpMaxE = 256;
 constexpr int kRpXTile = kRpTok * kRpBK * 2;     // 16 KB
 
 struct RpLayout {
-    int stage_bytes, bar_off, ids_off, cnt_off, misc_off, total;
+    int stages, stage_bytes, bar_off, ids_off, cnt_off, misc_off, total;
 };
 
 __host__ __device__ inline RpLayout rp_layout(int e_pad) {
     RpLayout L;
     L.stage_bytes = kRpXTile + e_pad * kRpBK * 2;
-    L.bar_off = kRpStages * L.stage_bytes;
-    L.ids_off = L.bar_off + (2 * kRpStages + 1) * 8;
+    const int fixed = (2 * kRpMaxStages + 1) * 8 + kRpTok * kRpMaxTopK * 4 + 4 * kRpMaxE * 4 + 16 + 1024;
+    L.stages = (kRpSmemLimit - fixed) / L.stage_bytes;
+    if (L.stages > kRpMaxStages) L.stages = kRpMaxStages;
+    L.bar_off = L.stages * L.stage_bytes;
+    L.ids_off = L.bar_off + (2 * kRpMaxStages + 1) * 8;
     L.cnt_off = L.ids_off + kRpTok * kRpMaxTopK * 4;
     L.misc_off = L.cnt_off + 4 * kRpMaxE * 4;
     L.total = L.misc_off + 16 + 1024;   // + slack for the 1024-B alignment of the base
@@ -70,9 +76,10 @@ route_project_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bar_off);
+    const int NS = Ly.stages;
     uint64_t* full = bars;
-    uint64_t* empty = bars + kRpStages;
-    uint64_t* done = bars + 2 * kRpStages;
+    uint64_t* empty = bars + kRpMaxStages;
+    uint64_t* done = bars + 2 * kRpMaxStages;
     int32_t* s_ids = reinterpret_cast<int32_t*>(smem + Ly.ids_off);
     int32_t* s_cnt = reinterpret_cast<int32_t*>(smem + Ly.cnt_off);    // [4 warps][kRpMaxE]
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc_off);
@@ -84,7 +91,7 @@ route_project_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
     const uint32_t ncols = e_pad <= 32 ? 32 : e_pad <= 64 ? 64 : e_pad <= 128 ? 128 : 256;
 
     if (tid == 0) {
-        for (int s = 0; s < kRpStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -111,9 +118,9 @@ route_project_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
         const uint32_t bytes = static_cast<uint32_t>(Ly.stage_bytes);
         int issued = 0;
         for (int ks = 0; ks < nk; ++ks, ++issued) {
-            const int s = ks % kRpStages;
-            const uint32_t ph = (ks / kRpStages) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1, s_abort)) { ok = false; break; }
+            const int s = ks % NS;
+            const uint32_t ph = (ks / NS) & 1;
+            if (!mbar_wait_spin(&empty[s], ph ^ 1, s_abort)) { ok = false; break; }
             uint8_t* st = smem + s * Ly.stage_bytes;
             mbar_arrive_expect_tx(&full[s], bytes);
             tma_load_2d(st, &tmap_x, &full[s], ks * kRpBK, tok0);
@@ -122,15 +129,15 @@ route_project_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
         if (!ok) {
             *s_abort = 1;
             record_status(status, MXFP4_ERR_TIMEOUT);
-            for (int i = issued > kRpStages ? issued - kRpStages : 0; i < issued; ++i)
-                mbar_wait(&full[i % kRpStages], (i / kRpStages) & 1, s_never);
+            for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
+                mbar_wait(&full[i % NS], (i / NS) & 1, s_never);
         }
     } else if (tid == 32) {
         // ---------------- MMA issuer: D[128 x e_pad] += x_tile . W_tile^T, K = 16 per MMA
         const uint32_t idesc = idesc_bf16_f32(kRpTok, e_pad);
         for (int ks = 0; ks < nk; ++ks) {
-            const int s = ks % kRpStages;
-            if (!mbar_wait(&full[s], (ks / kRpStages) & 1, s_abort)) { ok = false; break; }
+            const int s = ks % NS;
+            if (!mbar_wait_spin(&full[s], (ks / NS) & 1, s_abort)) { ok = false; break; }
             tc_fence_after();
             const uint32_t xa = smem_u32(smem + s * Ly.stage_bytes);
             const uint32_t wa = xa + kRpXTile;
@@ -151,7 +158,7 @@ route_project_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
     // ---------------- top-k epilogue: thread tid = token tok0 + tid (TMEM lane tid)
     // (waited for even after an abort: the MMAs in flight must finish before TMEM is
     // read or released, and the issuer commits `done` on every path)
-    const bool got = mbar_wait(done, 0, s_never);
+    const bool got = mbar_wait_spin(done, 0, s_never);
     if (!__all_sync(0xFFFFFFFFu, got)) {
         *s_abort = 1;
         record_status(status, MXFP4_ERR_TIMEOUT);

@@ -40,7 +40,7 @@ from . import build as _build
 __all__ = [
     "E2M1_GRID", "FLOOR", "CEIL", "e2m1_magnitude", "bf16_to_f64", "f64_to_bf16",
     "quantize", "dequantize_bf16", "dequantize_f64", "route", "gemm_w4a16",
-    "gemm_w4a4", "moe_mlp", "moe_down", "silu", "router_logits",
+    "gemm_w4a4", "moe_mlp", "moe_down", "silu", "router_logits", "moe_mlp_dense",
 ]
 
 FLOOR = 0
@@ -326,5 +326,31 @@ def moe_down(h_bits, logits, top_k, w2_codes, w2_scales, mode: str = "w4a16", to
         hb = h_bits[rows, slots]
         h = _fake_quant_bf16(hb) if mode == "w4a4" else bf16_to_f64(hb)
         y = h @ _deq_weights(w2_codes[e], w2_scales[e]).T
+        np.add.at(out, rows, w[rows, slots][:, None] * y)
+    return out
+
+
+def moe_mlp_dense(x_bits, logits, top_k, w13_bits, w2_bits, tokens=None):
+    """The expert MLP of ``moe_mlp`` with bf16 expert weights instead of MXFP4 ones
+    (the pages' bf16 fallback, [P4] "Native Support in transformers"): w13 bf16 bits
+    [E, 2I, H] (rows [0, I) gate, [I, 2I) up), w2 bf16 bits [E, H, I]; for each token
+    t and slot j with expert e (``route``): g, u = x_t W13[e]^T split, h =
+    bf16(SiLU(g) * u), y = h W2[e]^T; out_t = sum_j w_tj * y_j, fp64, unrounded."""
+    x_bits = _as_bf16_bits(x_bits)
+    T, H = x_bits.shape
+    E, twoI, _ = w13_bits.shape
+    I = twoI // 2
+    r = route(logits, top_k)
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    xf = bf16_to_f64(x_bits[tok])
+    ids, w = r["ids"][tok], r["w"][tok]
+    out = np.zeros((tok.size, H), dtype=np.float64)
+    for e in np.unique(ids):
+        rows, slots = np.nonzero(ids == e)
+        W13 = bf16_to_f64(_as_bf16_bits(w13_bits[e]))
+        g = xf[rows] @ W13[:I].T
+        u = xf[rows] @ W13[I:].T
+        h = bf16_to_f64(f64_to_bf16(silu(g) * u))
+        y = h @ bf16_to_f64(_as_bf16_bits(w2_bits[e])).T
         np.add.at(out, rows, w[rows, slots][:, None] * y)
     return out

@@ -134,3 +134,23 @@ def test_gemm_w4a4_equals_w4a16_on_grid_activations():
     y4 = _run(x, wc, ws, mx.W4A4)
     y16 = _run(x, wc, ws, mx.W4A16)
     assert_close_tol(y4, y16, what="w4a4 vs w4a16 on grid")
+
+
+@pytest.mark.parametrize("M", [130, 400])   # 128- and 192-row token tiles (ALU dequantization)
+@pytest.mark.parametrize("scales", ["subnormal", "mixed"])
+def test_gemm_large_tiles_every_dequant_route(M, scales):
+    """Large token tiles dequantize without the LUT: an f16 conversion, a shift and one
+    bf16x2 multiply for scale bytes 2..142, the exact fp32 route otherwise.  Weights with
+    random codes and scale bytes on both sides of that boundary (or all subnormal)."""
+    K, N = 512, 256
+    g = torch.Generator().manual_seed(M + (0 if scales == "subnormal" else 1))
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    wc = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8).numpy()
+    if scales == "subnormal":   # 30% of the blocks at S = 0, 1 (subnormal weights), the rest normal
+        tiny = torch.rand((N, K // 32), generator=g) < 0.3
+        ws = torch.where(tiny, torch.randint(0, 2, (N, K // 32), generator=g),
+                         torch.randint(120, 128, (N, K // 32), generator=g)).to(torch.uint8).numpy()
+    else:
+        ws = torch.randint(120, 160, (N, K // 32), generator=g, dtype=torch.uint8).numpy()  # both routes
+    y = _run(x, wc, ws)
+    assert_close_tol(y, oracle.gemm_w4a16(bits_of(x), wc, ws), what=f"gemm {M}x{K}x{N} scales {scales}")

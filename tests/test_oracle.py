@@ -400,6 +400,26 @@ def test_router_logits_bruteforce():
     assert np.array_equal(oracle.router_logits(onehot, wb)[0], wf[:, 17])
 
 
+def test_moe_mlp_dense_with_dequantized_weights_is_moe_mlp():
+    # the bf16-weight layer's reference, fed the bf16 values of MXFP4 weights, is the
+    # (pinned) MXFP4 layer bit for bit; a swapped gate/up or a missing weight would not be
+    g = torch.Generator().manual_seed(25)
+    T, H, I, E, k = 11, 64, 96, 4, 2
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    logits = torch.randn(T, E, generator=g).numpy()
+    q13 = [oracle.quantize((torch.randn(2 * I, H, generator=g) * 0.1).numpy()) for _ in range(E)]
+    q2 = [oracle.quantize((torch.randn(H, I, generator=g) * 0.1).numpy()) for _ in range(E)]
+    w13c, w13s = np.stack([a for a, _ in q13]), np.stack([b for _, b in q13])
+    w2c, w2s = np.stack([a for a, _ in q2]), np.stack([b for _, b in q2])
+    ref = oracle.moe_mlp(xb, logits, k, w13c, w13s, w2c, w2s)
+    w13b = oracle.dequantize_bf16(w13c, w13s)
+    w2b = oracle.dequantize_bf16(w2c, w2s)
+    assert np.array_equal(oracle.moe_mlp_dense(xb, logits, k, w13b, w2b), ref)
+    swapped = np.concatenate([w13b[:, I:], w13b[:, :I]], axis=1)
+    assert not np.allclose(oracle.moe_mlp_dense(xb, logits, k, swapped, w2b), ref)
+
+
 # ----------------------------------------------------------------- GEMM
 
 def test_gemm_bruteforce():

@@ -98,3 +98,26 @@ def test_expert_parallel_layer_on_one_nccl_rank(mode):
     assert mx.mxfp4_get_device_status() == 0
     assert trace["send_rows"] == [T * k] and trace["recv_rows"] == [T * k]
     assert np.array_equal(bits_of(out), bits_of(ref))
+
+
+# ---------------------------------------------------------------- bf16-weight comparison layer
+
+def _bf16_layer(T, H, I, E, k, seed):
+    cfg = inputs.MoEConfig("bf16w", seed=seed, T=T, E=E, top_k=k, H=H, I=I, w_std=0.05)
+    x, logits = inputs.moe_activations(cfg)
+    w13 = torch.stack([inputs.expert_weights(cfg, e)[0] for e in range(E)]).to(torch.bfloat16)
+    w2 = torch.stack([inputs.expert_weights(cfg, e)[1] for e in range(E)]).to(torch.bfloat16)
+    return x, logits, w13, w2
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [(5, 128, 64, 4, 2), (37, 192, 128, 8, 2), (300, 256, 320, 32, 4),
+                                       (64, 2880, 2880, 32, 4), (400, 320, 256, 8, 2), (700, 512, 384, 8, 3),
+                                       (2048, 256, 192, 4, 2)])
+def test_bf16_weight_layer_against_oracle(T, H, I, E, k):
+    x, logits, w13, w2 = _bf16_layer(T, H, I, E, k, seed=T + H)
+    out = mx.moe_bf16_mlp(x.to(DEV), logits.to(DEV), k, w13.to(DEV), w2.to(DEV))
+    torch.cuda.synchronize()
+    assert mx.mxfp4_get_device_status() == 0
+    ref = oracle.moe_mlp_dense(bits_of(x), logits.numpy(), k, bits_of(w13), bits_of(w2))
+    from helpers import assert_close_tol, f64_of
+    assert_close_tol(f64_of(out), ref, what=f"bf16-weight layer T={T} H={H} I={I} E={E} k={k}")
