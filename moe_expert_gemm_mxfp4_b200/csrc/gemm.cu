@@ -81,12 +81,6 @@ struct Cfg {
     static constexpr int kActUnit = kLock ? kSub * kActStage : kActStage;   // bytes per ring slot
     static constexpr int kMaxActStages = kLock ? 4 : (TT == 1 ? (NT > 128 ? 4 : 5) : kSub);
     static constexpr int kChunk = kAccCols < 32 ? kAccCols : 32;   // epilogue columns per TMEM load
-    // Dequantize with the ALU (no LUT) for the large token tiles: there the MMA already
-    // reads and the TMA writes the whole token tile through shared memory every stage,
-    // and the LUT's reads would add a third of that again; the ALU route needs more
-    // instructions per byte, which the small tiles (weights streamed at HBM rate) can't
-    // afford but the large ones (NT tokens per weight) can.
-    static constexpr bool kAluDequant = NT >= 128;
     static_assert(kActTile % 1024 == 0, "activation tiles must keep 1024-B alignment");
     static_assert(kAccCols <= kACol, "accumulators overlap the A slots");
     static_assert(!kLock || kGrp == kSub, "the chunked activation ring follows groups of kSub stages");
@@ -171,42 +165,6 @@ __device__ __forceinline__ void dequant_block16(uint4 c, uint32_t S, uint32_t lu
                 const uint32_t a = prmt(w[i], lut_lane, 0x7604u | (j << 4));
                 out[4 * i + j] = bmul2(lds32(a), sf);
             }
-        }
-    } else {
-        const float sc = e8m0_f32(S);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) out[4 * i + j] = dequant_byte_exact((w[i] >> (8 * j)) & 0xFFu, sc);
-    }
-}
-
-// 4 code bytes -> 4 f16x2 words holding their E2M1 values exactly (low nibble in the
-// low half): the hardware E2M1 -> f16 conversion.
-__device__ __forceinline__ void cvt_e2m1x8_f16(uint32_t w, uint32_t* o) {
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
-        : "r"(w));
-}
-
-// The same 16 code bytes -> 16 bf16x2 words as dequant_block16, without the LUT (no
-// shared-memory traffic).  An E2M1 value in f16 has its magnitude in bits 9-14 only, so
-// shifting the magnitude right by 3 (sign kept) gives the bf16 pattern of the value
-// times 2^-112; one exact bf16x2 multiply by 2^(S-15) then gives value x 2^(S-127), for
-// S in [2, 142] (normal operands and products).  Other S take the exact fp32 route.
-__device__ __forceinline__ void dequant_block16_alu(uint4 c, uint32_t S, uint32_t* out) {
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    if (S - 2u <= 140u) {
-        const uint32_t sf = (S + 112u) * 0x00800080u;   // bf16x2 {2^(S-15), 2^(S-15)}
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t h[4];
-            cvt_e2m1x8_f16(w[i], h);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                out[4 * i + j] = bmul2(((h[j] & 0x7FFF7FFFu) >> 3) | (h[j] & 0x80008000u), sf);
         }
     } else {
         const float sc = e8m0_f32(S);
@@ -528,13 +486,8 @@ grouped_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,
                             const uint4 c0 = lds128(row_addr + (((2u * j) ^ sw) << 4));
                             const uint4 c1 = lds128(row_addr + (((2u * j + 1u) ^ sw) << 4));
                             uint32_t out[32];
-                            if (C::kAluDequant) {
-                                dequant_block16_alu(c0, sc & 0xFFu, out);
-                                dequant_block16_alu(c1, sc >> 8, out + 16);
-                            } else {
-                                dequant_block16(c0, sc & 0xFFu, lut_lane, out);
-                                dequant_block16(c1, sc >> 8, lut_lane, out + 16);
-                            }
+                            dequant_block16(c0, sc & 0xFFu, lut_lane, out);
+                            dequant_block16(c1, sc >> 8, lut_lane, out + 16);
                             tmem_st_x32(tmem_lane + (a.idx * C::kGrp + jg) * 32, out);
                             const int xs = xr.idx;      // kLock: the group's chunk
                             const uint32_t xph = xr.ph;

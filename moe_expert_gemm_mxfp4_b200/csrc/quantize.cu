@@ -222,73 +222,10 @@ __device__ __forceinline__ void ring_release(Ring& r, int st) {
 }
 
 // ---------------------------------------------------------------- bf16 -> MXFP4
-// Chunk = 256 blocks (16 KB of bf16).  Consumer warp w converts blocks
-// 32w .. 32w+31 of the chunk: lane l reads vectors 32j + l (j = 0..3) of the
-// warp's 2 KB, so block 8j + l/4 lives on lanes 4(l/4) .. +3, and each lane
-// writes the 4 code bytes of its vector (a warp store covers 128 contiguous
-// bytes).  The 32 scale bytes are gathered by shuffles so that lane l stores
-// block l's.
-constexpr int kChunkBlocks = 256;
-
-__global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
-quantize_bf16_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint32_t* __restrict__ codes,
-                     uint8_t* __restrict__ scales, int rule, unsigned* status) {
-    constexpr int kStageBytes = kChunkBlocks * 64;
-    constexpr int kStages = kRingSmemBytes / kStageBytes;   // 6
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ Ring ring;
-    ring_init(ring, kStages);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t n_chunks = (n_blocks + kChunkBlocks - 1) / kChunkBlocks;
-    if (warp == kRingConsumerWarps) {
-        if (lane == 0)
-            ring_produce(ring, kStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
-                const int64_t nb = min(static_cast<int64_t>(kChunkBlocks), n_blocks - c * kChunkBlocks);
-                const uint32_t bytes = static_cast<uint32_t>(nb * 64);
-                mbar_arrive_expect_tx(bar, bytes);
-                bulk_load(smem + st * kStageBytes, x + c * kStageBytes, bytes, bar);
-            }, status);
-        return;
-    }
-    int st = 0;
-    uint32_t ph = 0;
-    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
-        if (!ring_wait_full(ring, st, ph, status)) break;
-        const uint4* src = reinterpret_cast<const uint4*>(smem + st * kStageBytes) + warp * 128;
-        uint4 v[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = src[32 * j + lane];
-        ring_release(ring, st);
-        const int64_t blk0 = c * kChunkBlocks + warp * 32;   // first block of this warp
-        uint32_t mine = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t am = amax8_bf16(v[j]);
-            am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-            am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
-            const bool nf = am >= 0x7F80u;
-            const int s = block_exp_bf16(am, rule);
-            const uint32_t cw = nf ? 0u : quant8_bf16(v[j], inv_pow2(s));
-            const uint32_t S = nf ? 0xFFu : static_cast<uint32_t>(s + 127);
-            const int64_t blk = blk0 + 8 * j + (lane >> 2);
-            if (blk < n_blocks) __stcs(codes + blk0 * 4 + 32 * j + lane, cw);
-            // block 8j + q (q = 0..7) lives on lanes 4q .. 4q+3; lane 8j + q takes its scale
-            const uint32_t got = __shfl_sync(0xFFFFFFFFu, S, (lane & 7) * 4);
-            if ((lane >> 3) == j) mine = got;
-        }
-        if (blk0 + lane < n_blocks) scales[blk0 + lane] = static_cast<uint8_t>(mine);
-        if (++st == kStages) {
-            st = 0;
-            ph ^= 1u;
-        }
-    }
-}
-
-// Same conversion, fed by plain 128-bit loads instead of the bulk-copy ring: warp u
-// of the grid converts 32-block units u, u + n_warps, ... (2 KB of bf16 each, read
-// as four fully coalesced 512-byte warp loads, non-allocating in L1), two units per
-// iteration so that 8 loads per lane are in flight.  Lane and block mapping and the
-// stores are those of quantize_bf16_kernel.
+// Plain 128-bit loads (no bulk-copy ring): warp u of the grid converts 32-block
+// units u, u + n_warps, ... (2 KB of bf16 each, read as four fully coalesced
+// 512-byte warp loads, non-allocating in L1), two units per iteration so that 8
+// loads per lane are in flight.
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -297,6 +234,10 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     return v;
 }
 
+// One 32-block unit held as v[j] = vector 32j + lane of the unit's 2 KB: block
+// 8j + l/4 lives on lanes 4(l/4) .. +3, each lane writes the 4 code bytes of its
+// vector (a warp store covers 128 contiguous bytes), and the 32 scale bytes are
+// gathered by shuffles so that lane l stores block l's.
 __device__ __forceinline__ void quant_unit_bf16(const uint4 (&v)[4], int64_t blk0, int64_t n_blocks, int lane,
                                                 uint32_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                 int rule) {
@@ -319,36 +260,36 @@ __device__ __forceinline__ void quant_unit_bf16(const uint4 (&v)[4], int64_t blk
 }
 
 constexpr int kLsuThreads = 256;
-constexpr int kLsuUnits = 4;   // 32-block units in flight per warp (16 loads per lane)
 
-// Warp w of the grid converts the contiguous range of units [w * n / W, (w + 1) * n / W)
-// (W warps, n units: every warp gets the same count to within one), kLsuUnits at a
-// time with all their loads issued before any conversion.
 __global__ void __launch_bounds__(kLsuThreads)
 quantize_bf16_lsu_kernel(const uint4* __restrict__ x, int64_t n_blocks, uint32_t* __restrict__ codes,
                          uint8_t* __restrict__ scales, int rule) {
     const int lane = threadIdx.x & 31;
-    const int64_t w = (static_cast<int64_t>(blockIdx.x) * kLsuThreads + threadIdx.x) >> 5;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * kLsuThreads + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * kLsuThreads) >> 5;
     const int64_t n_units = (n_blocks + 31) / 32;
-    const int64_t u_end = (w + 1) * n_units / nw;
     const int64_t n_vec = n_blocks * 4;   // 16-byte vectors of input
-    for (int64_t u = w * n_units / nw; u < u_end; u += kLsuUnits) {
-        uint4 v[kLsuUnits][4];
+    for (int64_t u = w0; u < n_units; u += 2 * nw) {
+        const int64_t u2 = u + nw;
+        uint4 a[4], b[4];
 #pragma unroll
-        for (int k = 0; k < kLsuUnits; ++k)
+        for (int j = 0; j < 4; ++j) {
+            const int64_t i = u * 128 + 32 * j + lane;
+            a[j] = i < n_vec ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int64_t i = (u + k) * 128 + 32 * j + lane;
-                v[k][j] = (u + k < u_end && i < n_vec) ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-        for (int k = 0; k < kLsuUnits; ++k)
-            if (u + k < u_end) quant_unit_bf16(v[k], (u + k) * 32, n_blocks, lane, codes, scales, rule);
+        for (int j = 0; j < 4; ++j) {
+            const int64_t i = u2 * 128 + 32 * j + lane;
+            b[j] = (u2 < n_units && i < n_vec) ? ld_stream(x + i) : make_uint4(0, 0, 0, 0);
+        }
+        quant_unit_bf16(a, u * 32, n_blocks, lane, codes, scales, rule);
+        if (u2 < n_units) quant_unit_bf16(b, u2 * 32, n_blocks, lane, codes, scales, rule);
     }
 }
 
 // ---------------------------------------------------------------- fp32 -> MXFP4
+constexpr int kChunkBlocks = 256;
+
 // Chunk = 256 blocks (32 KB of fp32).  Consumer warp w converts blocks
 // 32w .. 32w+31: step j (0..7) reads vectors 32j + l, i.e. block 4j + l/8, a
 // block spanning 8 lanes; each lane produces 2 code bytes.
@@ -524,14 +465,8 @@ cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t col
     } else {
         (void)status;
         const int64_t n_units = (n_blocks + 31) / 32;
-        // one wave of resident CTAs (each warp then owns an equal contiguous range), fewer
-        // when there are not kLsuUnits units per warp
-        int per_sm = 0;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_bf16_lsu_kernel, kLsuThreads, 0)) !=
-            cudaSuccess)
-            return e;
-        int64_t g = (n_units + kLsuUnits * (kLsuThreads / 32) - 1) / (kLsuUnits * (kLsuThreads / 32));
-        const int64_t cap = static_cast<int64_t>(sm_count) * (per_sm > 0 ? per_sm : 1);
+        int64_t g = (n_units + 2 * (kLsuThreads / 32) - 1) / (2 * (kLsuThreads / 32));
+        const int64_t cap = static_cast<int64_t>(sm_count) * 8;
         if (g > cap) g = cap;
         quantize_bf16_lsu_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), kLsuThreads, 0, stream>>>(
             static_cast<const uint4*>(x), n_blocks, reinterpret_cast<uint32_t*>(codes), scales, rule);
