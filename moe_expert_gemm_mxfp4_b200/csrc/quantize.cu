@@ -7,18 +7,21 @@
 // element, Inf/NaN blocks -> scale 0xFF) are documented in include/mxfp4.h.
 //
 // Layout of the work: the input is treated as a flat array of 32-element blocks
-// (cols % 32 == 0, so blocks never straddle rows), cut into chunks of
-// consecutive blocks.  Each CTA is persistent over chunks c = blockIdx.x,
-// blockIdx.x + gridDim.x, ...: one producer thread streams its chunks into a
-// ring of shared-memory stages with cp.async.bulk (completion counted on an
-// mbarrier per stage), so that a whole ring of bytes per CTA is in flight from
-// HBM; eight consumer warps convert a stage and release it.  Quantize: 128-bit
-// shared-memory reads spread each block over 4 lanes (bf16) or 8 lanes (fp32);
-// the block amax is a shuffle reduction over those lanes; the scale is pure
-// integer work on the amax bit pattern; |v| / 2^s is an exact power-of-two
-// product in fp32 and the E2M1 rounding is the hardware
-// cvt.rn.satfinite.e2m1x2.f32 (round-to-nearest-even, saturating at 6).
-// Dequantize: each lane expands 4 code bytes to 8 bf16 values exactly.
+// (cols % 32 == 0, so blocks never straddle rows).
+//   bf16 -> MXFP4 and MXFP4 -> bf16 stream with plain 128-bit (codes: 32-bit)
+//   loads, non-allocating in L1: each warp of the grid takes 32-block units in a
+//   grid-stride walk, two at a time, so that every lane has its loads of two
+//   units in flight before it computes.
+//   fp32 -> MXFP4 (weights, off the hot path) runs a ring of cp.async.bulk stages
+//   per persistent CTA: one producer thread streams chunks of consecutive blocks
+//   into shared memory (completion counted on an mbarrier per stage) and eight
+//   consumer warps convert and release them.
+// Quantize: each block is spread over 4 lanes (bf16) or 8 lanes (fp32); the block
+// amax is a shuffle reduction over those lanes; the scale is pure integer work on
+// the amax bit pattern; |v| / 2^s is an exact power-of-two product in fp32 and the
+// E2M1 rounding is the hardware cvt.rn.satfinite.e2m1x2.f32 (round-to-nearest-even,
+// saturating at 6).  Dequantize: the hardware E2M1 -> f16 conversion, a shift into
+// a bf16 pattern and one exact bf16x2 multiply by the block scale per code pair.
 #include "common.cuh"
 #include "internal.h"
 
@@ -127,26 +130,28 @@ __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
+// 2 E2M1 codes (one byte, low nibble first) -> their values as f16x2, exactly.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t o;
+    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(o) : "r"(byte));
+    return o;
 }
 
-// Dequantize one code word through the lane-replicated LUT of bf16 pairs (entry
-// (b, lane) at lut + b * 256 + lane * 4): for S in [2, 254] the LUT value times
-// 2^(S-127) is one exact bf16x2 product (normal operands; a product past the
-// bf16 range rounds to Inf as round-to-nearest-even does).  S in {0, 1, 255} takes
-// the exact fp32 route.
-__device__ __forceinline__ uint4 dequant8_lut(uint32_t cw, uint32_t S, uint32_t lut_lane) {
-    if (S - 2u > 252u) return dequant8(cw, S);
-    const uint32_t sf = S * 0x00800080u;   // bf16x2 {2^(S-127), 2^(S-127)}
-    uint4 o;
-    o.x = bmul2(lds32(prmt(cw, 0u, 0x4404u) + lut_lane), sf);
-    o.y = bmul2(lds32(prmt(cw, 0u, 0x4414u) + lut_lane), sf);
-    o.z = bmul2(lds32(prmt(cw, 0u, 0x4424u) + lut_lane), sf);
-    o.w = bmul2(lds32(prmt(cw, 0u, 0x4434u) + lut_lane), sf);
-    return o;
+// Dequantize one code word (8 codes) with the block's scale byte S -> 8 bf16.
+// An E2M1 value as f16 has a 1-bit mantissa; shifting the f16 magnitude right by 3
+// (sign kept) gives the bf16 pattern of the same value times 2^-112, and one exact
+// bf16x2 multiply by 2^(S-15) then gives value x 2^(S-127): exact for S in [2, 142]
+// (normal operands and products).  Other S take the exact fp32 route.
+__device__ __forceinline__ uint4 dequant8_alu(uint32_t cw, uint32_t S) {
+    if (S - 2u > 140u) return dequant8(cw, S);
+    const uint32_t sf = (S + 112u) * 0x00800080u;   // bf16x2 {2^(S-15), 2^(S-15)}
+    uint32_t r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t h = e2m1x2_to_f16x2((cw >> (8 * j)) & 0xFFu);
+        r[j] = bmul2(((h & 0x7FFF7FFFu) >> 3) | (h & 0x80008000u), sf);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 // ---------------------------------------------------------------- bulk-copy ring
@@ -360,77 +365,42 @@ quantize_f32_kernel(const uint8_t* __restrict__ x, int64_t n_blocks, uint16_t* _
 }
 
 // ---------------------------------------------------------------- MXFP4 -> bf16
-// Chunk = 1024 blocks: 16 KB of codes and 1 KB of scales per stage.  One CTA per
-// SM with 16 consumer warps and the 64 KB lane-replicated LUT of bf16 pairs
-// (dequant8_lut); consumer thread i expands code words i + 512 m (m = 0..7) of the
-// chunk, so a warp's output is 512 contiguous bytes per store instruction.  The
-// last few scale bytes of a ragged final chunk (fewer than 16) are read from
-// global memory directly, since a bulk copy moves whole 16-byte units.
-constexpr int kDqChunkBlocks = 1024;
-constexpr int kDqWarps = 16;
-constexpr int kDqThreads = (kDqWarps + 1) * 32;
-constexpr int kDqLutBytes = 256 * 256;
-constexpr int kDqStages = 8;
-constexpr int kDqCodeBytes = kDqChunkBlocks * 16;
-constexpr int kDqStageBytes = kDqCodeBytes + kDqChunkBlocks;
-constexpr int kDqSmemBytes = kDqLutBytes + kDqStages * kDqStageBytes;
+// Plain streaming loads, like the bf16 quantize: warp u of the grid expands 32-block
+// units u, u + n_warps, ... two per iteration.  Lane l, step j (0..3) takes code word
+// 32j + l of the unit (block 8j + l/4, whose scale byte lane 8j + l/4 loaded and a
+// shuffle hands over) and stores output vector 32j + l: every warp access is a
+// contiguous 128-byte (codes) or 512-byte (output) run.
+constexpr int kDqThreads = 256;
+constexpr int kDqUnits = 2;
 
-__global__ void __launch_bounds__(kDqThreads, 1)
-dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                  int64_t n_blocks, uint4* __restrict__ out, unsigned* status) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ Ring ring;
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-    uint8_t* stages = smem + kDqLutBytes;
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-        const uint32_t b = static_cast<uint32_t>(i >> 5);
-        lut[(b << 6) | (i & 31)] = e2m1_bf16(b & 15u) | (e2m1_bf16(b >> 4) << 16);
-    }
-    ring_init(ring, kDqStages, kDqWarps);   // its __syncthreads also publishes the LUT
-    const int warp = threadIdx.x >> 5;
-    const int64_t n_chunks = (n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks;
-    if (warp == kDqWarps) {
-        if ((threadIdx.x & 31) == 0)
-            ring_produce(ring, kDqStages, n_chunks, [&](int st, int64_t c, uint64_t* bar) {
-                const int64_t nb = min(static_cast<int64_t>(kDqChunkBlocks), n_blocks - c * kDqChunkBlocks);
-                const uint32_t cb = static_cast<uint32_t>(nb * 16);
-                const uint32_t sb = static_cast<uint32_t>(nb & ~int64_t{15});
-                mbar_arrive_expect_tx(bar, cb + sb);
-                uint8_t* dst = stages + st * kDqStageBytes;
-                bulk_load(dst, codes + c * kDqCodeBytes, cb, bar);
-                if (sb) bulk_load(dst + kDqCodeBytes, scales + c * kDqChunkBlocks, sb, bar);
-            }, status);
-        return;
-    }
-    int st = 0;
-    uint32_t ph = 0;
-    const int tid = threadIdx.x;
-    const uint32_t lut_lane = smem_u32(lut) + (threadIdx.x & 31) * 4;
-    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
-        if (!ring_wait_full(ring, st, ph, status)) break;
-        const int64_t nb = min(static_cast<int64_t>(kDqChunkBlocks), n_blocks - c * kDqChunkBlocks);
-        const int nw = static_cast<int>(nb * 4);                 // code words in this chunk
-        const int sb = static_cast<int>(nb & ~int64_t{15});      // scales staged in shared memory
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(stages + st * kDqStageBytes);
-        const uint8_t* sc = stages + st * kDqStageBytes + kDqCodeBytes;
-        uint32_t w[8], S[8];
+__global__ void __launch_bounds__(kDqThreads, 8)
+dequantize_kernel(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                  int64_t n_blocks, uint4* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * kDqThreads + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * kDqThreads) >> 5;
+    const int64_t n_units = (n_blocks + 31) / 32;
+    for (int64_t u = w0; u < n_units; u += kDqUnits * nw) {
+        uint32_t cw[kDqUnits][4], sb[kDqUnits];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int i = tid + 32 * kDqWarps * m;
-            const int b = i >> 2;
-            w[m] = i < nw ? cw[i] : 0u;
-            S[m] = i < nw ? (b < sb ? sc[b] : __ldg(scales + c * kDqChunkBlocks + b)) : 127u;
-        }
-        ring_release(ring, st);
-        uint4* o = out + c * (kDqChunkBlocks * 4);
+        for (int k = 0; k < kDqUnits; ++k) {
+            const int64_t uk = u + k * nw;
+            sb[k] = uk < n_units && uk * 32 + lane < n_blocks ? static_cast<uint32_t>(__ldcs(scales + uk * 32 + lane)) : 0u;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int i = tid + 32 * kDqWarps * m;
-            if (i < nw) __stcs(o + i, dequant8_lut(w[m], S[m], lut_lane));
+            for (int j = 0; j < 4; ++j) {
+                const int64_t blk = uk * 32 + 8 * j + (lane >> 2);
+                cw[k][j] = uk < n_units && blk < n_blocks ? __ldcs(codes + uk * 128 + 32 * j + lane) : 0u;
+            }
         }
-        if (++st == kDqStages) {
-            st = 0;
-            ph ^= 1u;
+#pragma unroll
+        for (int k = 0; k < kDqUnits; ++k) {
+            const int64_t uk = u + k * nw;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t S = __shfl_sync(0xFFFFFFFFu, sb[k], 8 * j + (lane >> 2));
+                const int64_t blk = uk * 32 + 8 * j + (lane >> 2);
+                if (uk < n_units && blk < n_blocks) __stcs(out + uk * 128 + 32 * j + lane, dequant8_alu(cw[k][j], S));
+            }
         }
     }
 }
@@ -477,14 +447,14 @@ cudaError_t launch_quantize(const void* x, int is_f32, int64_t rows, int64_t col
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
                               int64_t cols, void* out, int sm_count, unsigned* status,
                               cudaStream_t stream) {
+    (void)status;   // no waits in this kernel
     const int64_t n_blocks = rows * (cols / 32);
-    const int64_t n_chunks = (n_blocks + kDqChunkBlocks - 1) / kDqChunkBlocks;
-    const int grid = static_cast<int>(n_chunks < sm_count ? n_chunks : sm_count);
-    cudaError_t e = cudaFuncSetAttribute(dequantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kDqSmemBytes);
-    if (e != cudaSuccess) return e;
-    dequantize_kernel<<<grid, kDqThreads, kDqSmemBytes, stream>>>(
-        codes, scales, n_blocks, reinterpret_cast<uint4*>(out), status);
+    const int64_t n_units = (n_blocks + 31) / 32;
+    int64_t g = (n_units + kDqUnits * (kDqThreads / 32) - 1) / (kDqUnits * (kDqThreads / 32));
+    const int64_t cap = static_cast<int64_t>(sm_count) * 16;   // two waves of 8 CTAs per SM
+    if (g > cap) g = cap;
+    dequantize_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), kDqThreads, 0, stream>>>(
+        reinterpret_cast<const uint32_t*>(codes), scales, n_blocks, reinterpret_cast<uint4*>(out));
     return cudaGetLastError();
 }
 
