@@ -560,7 +560,7 @@ mxfp4_status moe_mxfp4_route_project(const void* x_bf16, int64_t T, int64_t H, c
     int32_t *chunk_counts, *local_rank;
     mx::route_tmp_split(ws, T, E, &chunk_counts, &local_rank);
     cudaError_t e = mx::launch_route_project(tx, tw, T, H, E, top_k, ids, weights, chunk_counts,
-                                             local_rank, logits_out, d->status, s);
+                                             local_rank, logits_out, d->sm_count, d->status, s);
     if (e != cudaSuccess) return cuda_fail(e);
     e = mx::launch_route_finish(T, E, top_k, ids, weights, counts, offsets, perm, inv, nullptr, nullptr,
                                 ws, nullptr, 0, nullptr, nullptr, 0, nullptr, d->sm_count, s);

@@ -59,11 +59,11 @@ cudaError_t launch_route_finish(int64_t T, int64_t E, int top_k, const int32_t* 
                                 int64_t row_bytes, void* x_sorted, const void* xs, int64_t xs_row_bytes,
                                 void* xs_sorted, int sm_count, cudaStream_t stream);
 void route_tmp_split(void* tmp, int64_t T, int64_t E, int32_t** chunk_counts, int32_t** local_rank);
-int route_project_smem_bytes(int64_t E);
+int route_project_smem_bytes(int64_t E, int64_t H, int cluster_size);
 cudaError_t launch_route_project(const CUtensorMap& tmap_x, const CUtensorMap& tmap_w, int64_t T,
                                  int64_t H, int64_t E, int top_k, int32_t* ids, float* weights,
                                  int32_t* chunk_counts, int32_t* local_rank, float* logits_out,
-                                 unsigned* status, cudaStream_t stream);
+                                 int sm_count, unsigned* status, cudaStream_t stream);
 cudaError_t launch_gather_rows(const void* src, int64_t n_src, int64_t row_bytes, const int32_t* idx,
                                int64_t n, int div, void* dst, int sm_count, unsigned* status,
                                cudaStream_t stream);

@@ -137,3 +137,23 @@ def test_route_project_ties_resolve_to_lower_ids():
     torch.cuda.synchronize()
     ro = oracle.route(r["logits"].cpu().numpy(), k)
     assert np.array_equal(r["ids"].cpu().numpy(), ro["ids"])
+
+
+def test_route_project_zero_tokens_tie_across_signed_zeros():
+    # a zero token's logits are all zeros, some of them -0 (negative weights): +0 and
+    # -0 are equal logits, so the lowest ids win and the weights are uniform
+    T, H, E, k = 40, 256, 32, 4
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    x[::3] = 0.0
+    w = (torch.randn(E, H, generator=g) * H ** -0.5).to(torch.bfloat16)
+    r = mx.moe_mxfp4_route_project(x.to(DEV), w.to(DEV), k, logits_out=True)
+    torch.cuda.synchronize()
+    assert mx.mxfp4_get_device_status() == 0
+    ids, wts = r["ids"].cpu().numpy(), r["weights"].cpu().numpy()
+    for t in range(0, T, 3):
+        assert np.all(r["logits"].cpu().numpy()[t] == 0.0)
+        assert list(ids[t]) == list(range(k)), (t, ids[t])
+        assert np.allclose(wts[t], 1.0 / k, rtol=1e-6)
+    ro = oracle.route(r["logits"].cpu().numpy(), k)
+    assert np.array_equal(ids, ro["ids"])
