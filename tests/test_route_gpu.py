@@ -106,9 +106,11 @@ def _check_project(x, w, k, what):
     return clear.mean()
 
 
+# the K split runs over clusters of 1 (H = 64, or T large enough to fill the SMs with
+# tiles: T = 10000), 2, 4 (E > 64) and 8 CTAs
 @pytest.mark.parametrize("T,H,E,k", [(1, 64, 1, 1), (37, 128, 8, 2), (50, 192, 20, 3), (130, 256, 256, 8),
                                      (200, 2880, 32, 4), (300, 2880, 128, 4), (1000, 2880, 32, 4),
-                                     (129, 640, 48, 6)])
+                                     (129, 640, 48, 6), (10000, 256, 16, 2)])
 def test_route_project_shapes(T, H, E, k):
     g = torch.Generator().manual_seed(T + H + E)
     x = torch.randn(T, H, generator=g).to(torch.bfloat16)
