@@ -174,3 +174,34 @@ def test_moe_decode_batch_256_tokens_full_size():
     assert 16 < _avg_rows(256, cfg.E, cfg.top_k) <= 32
     assert_close_tol(L.gpu(mx.W4A16), L.ref(), what="decode T=256 W4A16")
     L.check_w4a4(what="decode T=256 W4A4")
+
+
+# The large token tiles with every token compared at small H, I: 192-row tiles
+# (W4A16, experts averaging 320+ rows) and 128-row tiles (W4A4), ragged tails included.
+@pytest.mark.parametrize("mode,T,E,k", [(mx.W4A16, 1200, 4, 2), (mx.W4A16, 1000, 3, 1),
+                                        (mx.W4A4, 600, 4, 2), (mx.W4A4, 700, 5, 3)])
+def test_moe_large_token_tiles_all_tokens(mode, T, E, k):
+    L = Layer(_small(T, 128, 192, E, k, seed=T + E + k))
+    if mode == mx.W4A16:
+        assert _avg_rows(T, E, k) >= 320
+        assert_close_tol(L.gpu(mode), L.ref(), what=f"moe T={T} E={E} k={k} W4A16 (192-row tiles)")
+    else:
+        assert _avg_rows(T, E, k) > 64
+        L.check_w4a4(what=f"moe T={T} E={E} k={k} W4A4 (128-row tiles)")
+
+
+def test_moe_all_tokens_to_one_expert():
+    # a router bias so large that every token's top-1 is expert 0: one group holds all
+    # T rows (many token tiles), every other group is empty
+    cfg = inputs.MoEConfig("one_expert", seed=3, T=300, E=16, top_k=1, H=128, I=128,
+                           hot_experts=(0,), hot_bias=100.0, w_std=0.05)
+    L = Layer(cfg)
+    assert_close_tol(L.gpu(), L.ref(), what="all tokens to expert 0")
+
+
+def test_moe_widest_routing():
+    # the largest router the kernels take: 256 experts, top-8 (most experts hold a row
+    # or two, many none)
+    L = Layer(_small(96, 128, 64, 256, 8, seed=256))
+    assert_close_tol(L.gpu(), L.ref(), what="E=256 top-8")
+    L.check_w4a4(what="E=256 top-8 W4A4")
