@@ -136,12 +136,12 @@ def test_gemm_w4a4_equals_w4a16_on_grid_activations():
     assert_close_tol(y4, y16, what="w4a4 vs w4a16 on grid")
 
 
-@pytest.mark.parametrize("M", [130, 400])   # 128- and 192-row token tiles (ALU dequantization)
+@pytest.mark.parametrize("M", [130, 400])   # 128- and 192-row token tiles
 @pytest.mark.parametrize("scales", ["subnormal", "mixed"])
 def test_gemm_large_tiles_every_dequant_route(M, scales):
-    """Large token tiles dequantize without the LUT: an f16 conversion, a shift and one
-    bf16x2 multiply for scale bytes 2..142, the exact fp32 route otherwise.  Weights with
-    random codes and scale bytes on both sides of that boundary (or all subnormal)."""
+    """Large token tiles with weights of random codes and scale bytes: the fast path (LUT
+    value times 2^(S-127) in one bf16x2 multiply, S in 2..254) and the exact fp32 route
+    (S = 0, 1: subnormal weights) in the same tile."""
     K, N = 512, 256
     g = torch.Generator().manual_seed(M + (0 if scales == "subnormal" else 1))
     x = torch.randn(M, K, generator=g).to(torch.bfloat16)
@@ -154,3 +154,15 @@ def test_gemm_large_tiles_every_dequant_route(M, scales):
         ws = torch.randint(120, 160, (N, K // 32), generator=g, dtype=torch.uint8).numpy()  # both routes
     y = _run(x, wc, ws)
     assert_close_tol(y, oracle.gemm_w4a16(bits_of(x), wc, ws), what=f"gemm {M}x{K}x{N} scales {scales}")
+
+
+def test_gemm_largest_k():
+    # K = 7680, the largest contraction the W4A16 engine accepts (the tile's block
+    # scales are staged whole in shared memory next to the rings)
+    M, K, N = 40, 7680, 256
+    g = torch.Generator().manual_seed(7680)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    w = torch.randn(N, K, generator=g) * 0.02
+    wc, ws = oracle_quantize_weights(w)
+    y = _run(x, wc, ws)
+    assert_close_tol(y, oracle.gemm_w4a16(bits_of(x), wc, ws), what=f"gemm {M}x{K}x{N}")
