@@ -136,12 +136,12 @@ def test_gemm_w4a4_equals_w4a16_on_grid_activations():
     assert_close_tol(y4, y16, what="w4a4 vs w4a16 on grid")
 
 
-@pytest.mark.parametrize("M", [130, 400])   # 128- and 192-row token tiles
+@pytest.mark.parametrize("M", [20, 130, 400])   # 32-, 128- and 192-row token tiles
 @pytest.mark.parametrize("scales", ["subnormal", "mixed"])
-def test_gemm_large_tiles_every_dequant_route(M, scales):
-    """Large token tiles with weights of random codes and scale bytes: the fast path (LUT
-    value times 2^(S-127) in one bf16x2 multiply, S in 2..254) and the exact fp32 route
-    (S = 0, 1: subnormal weights) in the same tile."""
+def test_gemm_every_dequant_route(M, scales):
+    """Weights of random codes and scale bytes, so that the fast path (LUT value times
+    2^(S-127) in one bf16x2 multiply, S in 2..254) and the exact fp32 route (S = 0, 1:
+    subnormal weights) meet in the same tile, for each token tiling."""
     K, N = 512, 256
     g = torch.Generator().manual_seed(M + (0 if scales == "subnormal" else 1))
     x = torch.randn(M, K, generator=g).to(torch.bfloat16)
