@@ -39,6 +39,8 @@
 // TMEM: columns [0, 256) accumulators (TT*NT columns per buffer, double-buffered
 // when they fit), [256, 512) eight 32-column A slots (two sets of four).
 // Every mbarrier wait is time-bounded (MXFP4_ERR_TIMEOUT in the status word).
+#include <cmath>
+
 #include "gemm_common.cuh"
 
 namespace mx {
@@ -609,11 +611,14 @@ TokenTiling pick_token_tiling(int64_t rows, int64_t groups) {
     if (avg <= 16) return {16, 1};
     if (avg <= 32) return {32, 1};
     if (avg <= 64) return {64, 1};
-    // 192-row token tiles dequantize each weight tile once per 192 tokens instead of
-    // 128 (the dequantize work bounds the large-batch GEMM), at the cost of a ragged
-    // last tile per expert: worth it once experts average a few tiles
-    if (avg >= 320) return {192, 1};
-    return {128, 1};
+    // 128- or 192-row token tiles.  Each token tile dequantizes the expert's weight
+    // tiles once, and that bounds a tile's time, so a 192-row tile costs only ~1.25x a
+    // 128-row one (measured 1.23x with both at one tile per expert): take the size
+    // that needs fewer tiles, counted for an expert one standard deviation above the
+    // mean (routed counts spread about like the square root of the mean).
+    const double hi = static_cast<double>(avg) + std::sqrt(static_cast<double>(avg));
+    const double t128 = std::ceil(hi / 128.0), t192 = std::ceil(hi / 192.0);
+    return 1.25 * t192 < t128 ? TokenTiling{192, 1} : TokenTiling{128, 1};
 }
 
 // Largest K the kernel accepts: a tile's block scales must fit in shared memory
