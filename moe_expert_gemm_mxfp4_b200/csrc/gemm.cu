@@ -605,20 +605,28 @@ cudaError_t launch_mode(int nt, int tt, const CUtensorMap& tw, const CUtensorMap
 }  // namespace
 
 // Token tiling for `rows` activation rows spread over `groups` groups: NT rows per
-// MMA (16 .. 192).
+// MMA (16 .. 192).  Each token tile dequantizes the group's weight tiles once, and
+// that, not the MMA width, bounds a tile's time (at NT <= 64 an MMA costs the same
+// whatever its N).  So the cost of a tile grows only slowly with NT.  Measured on
+// the decode- and 120b-shaped layers, relative to a 16-row tile: 1.0 (32), 1.04
+// (64), 1.14 (128), 1.43 (192).  The launcher takes the NT with the least cost times
+// tiles, counted for a group one standard deviation above the mean (routed counts
+// spread about like the square root of the mean); ties go to the smaller tile.
 TokenTiling pick_token_tiling(int64_t rows, int64_t groups) {
     const int64_t avg = (rows + groups - 1) / (groups > 0 ? groups : 1);
-    if (avg <= 16) return {16, 1};
-    if (avg <= 32) return {32, 1};
-    if (avg <= 64) return {64, 1};
-    // 128- or 192-row token tiles.  Each token tile dequantizes the expert's weight
-    // tiles once, and that bounds a tile's time, so a 192-row tile costs only ~1.25x a
-    // 128-row one (measured 1.23x with both at one tile per expert): take the size
-    // that needs fewer tiles, counted for an expert one standard deviation above the
-    // mean (routed counts spread about like the square root of the mean).
     const double hi = static_cast<double>(avg) + std::sqrt(static_cast<double>(avg));
-    const double t128 = std::ceil(hi / 128.0), t192 = std::ceil(hi / 192.0);
-    return 1.25 * t192 < t128 ? TokenTiling{192, 1} : TokenTiling{128, 1};
+    constexpr int kNt[5] = {16, 32, 64, 128, 192};
+    constexpr double kCost[5] = {1.0, 1.0, 1.04, 1.14, 1.43};
+    int best = 0;
+    double best_cost = 0.0;
+    for (int i = 0; i < 5; ++i) {
+        const double c = kCost[i] * std::ceil(hi / kNt[i]);
+        if (i == 0 || c < best_cost) {
+            best = i;
+            best_cost = c;
+        }
+    }
+    return {kNt[best], 1};
 }
 
 // Largest K the kernel accepts: a tile's block scales must fit in shared memory

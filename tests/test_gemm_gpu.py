@@ -136,7 +136,7 @@ def test_gemm_w4a4_equals_w4a16_on_grid_activations():
     assert_close_tol(y4, y16, what="w4a4 vs w4a16 on grid")
 
 
-@pytest.mark.parametrize("M", [20, 130, 400])   # 32-, 128- and 192-row token tiles
+@pytest.mark.parametrize("M", [20, 100, 400])   # 32-, 128- and 192-row token tiles
 @pytest.mark.parametrize("scales", ["subnormal", "mixed"])
 def test_gemm_every_dequant_route(M, scales):
     """Weights of random codes and scale bytes, so that the fast path (LUT value times

@@ -151,11 +151,14 @@ def _avg_rows(T, E, k):
     return -(-T * k // E)
 
 
-# Token tiles of 32 and 64 rows (experts averaging 17-32 and 33-64 routed rows) with
-# both fused epilogues (SwiGLU, weighted), in W4A16 and W4A4, every token compared.
+# Token tiles of 32, 64 and 128 rows with both fused epilogues (SwiGLU, weighted), in
+# W4A16 and W4A4, every token compared.  The sizes land on the same tile in both engines:
+# W4A16 takes 32-row tiles for experts averaging 13-26 routed rows, 64-row ones for
+# 27-56 and 128-row ones for 57-117; W4A4 takes 32 up to 32 rows, 64 up to 64, then 128.
 @pytest.mark.parametrize("mode", [mx.W4A16, mx.W4A4])
-@pytest.mark.parametrize("T,H,I,nt", [(160, 384, 320, 32), (256, 256, 192, 32),
-                                      (400, 320, 256, 64), (512, 256, 384, 64)])
+@pytest.mark.parametrize("T,H,I,nt", [(160, 384, 320, 32), (208, 256, 192, 32),
+                                      (400, 320, 256, 64), (448, 256, 384, 64),
+                                      (640, 256, 192, 128)])
 def test_moe_mid_token_tiles_all_tokens(mode, T, H, I, nt):
     E, k = 32, 4
     assert nt // 2 < _avg_rows(T, E, k) <= nt
@@ -168,7 +171,8 @@ def test_moe_mid_token_tiles_all_tokens(mode, T, H, I, nt):
 
 def test_moe_decode_batch_256_tokens_full_size():
     """A 256-token decode batch of the gpt-oss-20b-shaped layer (experts average 32
-    routed rows, so the 32-row token tile), every token compared, W4A16 and W4A4."""
+    routed rows: 64-row token tiles in W4A16, 32-row ones in W4A4), every token
+    compared."""
     cfg = inputs.MOE_CONFIGS["moe_decode"]
     L = Layer(cfg, T=256)
     assert 16 < _avg_rows(256, cfg.E, cfg.top_k) <= 32
