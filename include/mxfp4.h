@@ -114,6 +114,15 @@ MXFP4_API mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K,
                         void* stream);
 MXFP4_API size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp4_mode mode);
 
+/* Token rows per work tile (the MMA's N side) that the grouped GEMMs take for `rows`
+ * activation rows spread over `groups` groups: one group in mxfp4_gemm, the experts in
+ * the MoE layer (rows = T * top_k).  W4A16: 16, 32, 64, 128 or 192, the size with the
+ * least measured tile cost times tiles for a group one standard deviation above the
+ * mean; W4A4: the smallest of 16, 32, 64, 128 that holds the mean.  A host query for
+ * tests and tuning: no CUDA call.  Returns 0 when rows < 1, groups < 1 or the mode is
+ * unknown.  No counterpart in the pages: the launch policy of the GEMMs above. */
+MXFP4_API int32_t mxfp4_token_tile_rows(int64_t rows, int64_t groups, mxfp4_mode mode);
+
 /* ---------------------------------------------------------------- routing
  * Per token t of router logits [T, E] fp32: the top_k experts ordered by
  * (logit descending, expert id ascending) -> ids int32 [T, top_k]; softmax over

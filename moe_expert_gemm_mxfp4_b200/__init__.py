@@ -23,6 +23,7 @@ from ._lib import (Mxfp4Error, Mxfp4LibraryMissing, SCALE_CEIL, SCALE_FLOOR, W4A
 
 __all__ = [
     "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_gemm_workspace_size",
+    "mxfp4_token_tile_rows",
     "moe_mxfp4_route", "moe_mxfp4_route_workspace_size", "moe_mxfp4_mlp",
     "moe_mxfp4_workspace_size", "moe_mxfp4_mlp_noalloc", "mxfp4_get_device_status",
     "mxfp4_selftest_wait_timeout", "mxfp4_selftest_mma_rate", "mxfp4_set_trace_events",
@@ -127,6 +128,11 @@ def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, out=None, stream
 
 def mxfp4_gemm_workspace_size(M, K, N, mode=W4A16) -> int:
     return int(_lib.load().mxfp4_gemm_workspace_size(M, K, N, int(mode)))
+
+
+def mxfp4_token_tile_rows(rows, groups=1, mode=W4A16) -> int:
+    """Token rows per work tile the grouped GEMMs take for `rows` rows over `groups` groups."""
+    return int(_lib.load().mxfp4_token_tile_rows(rows, groups, int(mode)))
 
 
 def mxfp4_gemm(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, mode: int = W4A16,

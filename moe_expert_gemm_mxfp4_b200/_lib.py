@@ -51,6 +51,7 @@ _SIGS = {
     "mxfp4_dequantize": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "mxfp4_gemm": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, ctypes.c_int, _vp, _sz, _vp]),
     "mxfp4_gemm_workspace_size": (_sz, [_i64, _i64, _i64, ctypes.c_int]),
+    "mxfp4_token_tile_rows": (_i32, [_i64, _i64, ctypes.c_int]),
     "moe_mxfp4_route": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_mxfp4_route_workspace_size": (_sz, [_i64, _i64, _i32]),
     "moe_mxfp4_route_project": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,

@@ -438,6 +438,13 @@ size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp4_mode mod
            align_up(static_cast<size_t>(M) * K / 32 + 16, 256);
 }
 
+int32_t mxfp4_token_tile_rows(int64_t rows, int64_t groups, mxfp4_mode mode) {
+    if (rows < 1 || groups < 1) return 0;
+    if (mode == MXFP4_W4A16) return mx::pick_token_tiling(rows, groups).nt;
+    if (mode == MXFP4_W4A4) return mx::pick_token_tiling_w4a4(rows, groups).nt;
+    return 0;
+}
+
 mxfp4_status mxfp4_gemm(const void* x_bf16, int64_t M, int64_t K, const uint8_t* w_codes,
                         const uint8_t* w_scales, int64_t N, void* y_bf16, mxfp4_mode mode,
                         void* ws, size_t ws_bytes, void* stream) {

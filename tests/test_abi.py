@@ -68,6 +68,41 @@ def test_gemm_argument_checks(lib):
     assert lib.mxfp4_gemm_workspace_size(8, 256, 512, 1) >= 8 * 256 // 2 + 8 * 256 // 32 + 16
 
 
+# Switch points of the W4A16 token-tiling rule: least tile cost x tiles (costs 1.0, 1.0,
+# 1.04, 1.14, 1.43 for 16- to 192-row tiles) for a group one standard deviation (the
+# square root of the mean) above the mean rows per group.
+W4A16_TILES = [(1, 16), (12, 16), (13, 32), (26, 32), (27, 64), (56, 64), (57, 128),
+               (117, 128), (118, 192), (178, 192), (179, 128), (240, 128), (241, 192),
+               (552, 192), (553, 128), (615, 128), (616, 192), (1024, 192)]
+
+
+@pytest.mark.parametrize("avg,nt", W4A16_TILES)
+def test_w4a16_token_tiles(lib, avg, nt):
+    assert lib.mxfp4_token_tile_rows(avg, 1, 0) == nt
+    # the mean is rows / groups, rounded up
+    assert lib.mxfp4_token_tile_rows(avg * 32 - 31, 32, 0) == nt
+    assert mx.mxfp4_token_tile_rows(avg * 32, 32) == nt
+
+
+def test_token_tile_rule_between_switch_points(lib):
+    """Between two listed switch points the choice does not change, and a brute-force
+    restatement of the rule agrees at every mean up to 2048."""
+    import math
+    cost = {16: 1.0, 32: 1.0, 64: 1.04, 128: 1.14, 192: 1.43}
+    for avg in range(1, 2049):
+        hi = avg + math.sqrt(avg)
+        want = min(cost, key=lambda n: (cost[n] * math.ceil(hi / n), n))
+        assert lib.mxfp4_token_tile_rows(avg, 1, 0) == want, avg
+
+
+def test_w4a4_token_tiles_and_invalid_queries(lib):
+    for avg, nt in [(1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64), (65, 128), (4096, 128)]:
+        assert lib.mxfp4_token_tile_rows(avg, 1, 1) == nt
+    assert lib.mxfp4_token_tile_rows(0, 1, 0) == 0
+    assert lib.mxfp4_token_tile_rows(8, 0, 0) == 0
+    assert lib.mxfp4_token_tile_rows(8, 1, 7) == 0
+
+
 def test_route_and_moe_argument_checks(lib):
     r = lib.moe_mxfp4_route
     assert r(A, 64, 32, 0, A, A, A, A, A, A, A, 1 << 20, N) == _lib.ERR_INVALID_ARG

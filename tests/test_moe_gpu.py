@@ -147,21 +147,16 @@ def test_moe_small_w4a4_all_tokens():
     L.check_w4a4(what="small W4A4")
 
 
-def _avg_rows(T, E, k):
-    return -(-T * k // E)
-
-
 # Token tiles of 32, 64 and 128 rows with both fused epilogues (SwiGLU, weighted), in
-# W4A16 and W4A4, every token compared.  The sizes land on the same tile in both engines:
-# W4A16 takes 32-row tiles for experts averaging 13-26 routed rows, 64-row ones for
-# 27-56 and 128-row ones for 57-117; W4A4 takes 32 up to 32 rows, 64 up to 64, then 128.
+# W4A16 and W4A4, every token compared.  The sizes land on the same tile in both engines
+# (the library's own tiling query says which).
 @pytest.mark.parametrize("mode", [mx.W4A16, mx.W4A4])
 @pytest.mark.parametrize("T,H,I,nt", [(160, 384, 320, 32), (208, 256, 192, 32),
                                       (400, 320, 256, 64), (448, 256, 384, 64),
                                       (640, 256, 192, 128)])
 def test_moe_mid_token_tiles_all_tokens(mode, T, H, I, nt):
     E, k = 32, 4
-    assert nt // 2 < _avg_rows(T, E, k) <= nt
+    assert mx.mxfp4_token_tile_rows(T * k, E, mode) == nt
     L = Layer(_small(T, H, I, E, k, seed=T + H))
     if mode == mx.W4A16:
         assert_close_tol(L.gpu(mode), L.ref(), what=f"moe T={T} E={E} (NT={nt}) W4A16")
@@ -175,22 +170,23 @@ def test_moe_decode_batch_256_tokens_full_size():
     compared."""
     cfg = inputs.MOE_CONFIGS["moe_decode"]
     L = Layer(cfg, T=256)
-    assert 16 < _avg_rows(256, cfg.E, cfg.top_k) <= 32
+    assert mx.mxfp4_token_tile_rows(256 * cfg.top_k, cfg.E, mx.W4A16) == 64
+    assert mx.mxfp4_token_tile_rows(256 * cfg.top_k, cfg.E, mx.W4A4) == 32
     assert_close_tol(L.gpu(mx.W4A16), L.ref(), what="decode T=256 W4A16")
     L.check_w4a4(what="decode T=256 W4A4")
 
 
-# The large token tiles with every token compared at small H, I: 192-row tiles
-# (W4A16, experts averaging 320+ rows) and 128-row tiles (W4A4), ragged tails included.
-@pytest.mark.parametrize("mode,T,E,k", [(mx.W4A16, 1200, 4, 2), (mx.W4A16, 1000, 3, 1),
+# The large token tiles with every token compared at small H, I: 192-row tiles (W4A16)
+# and 128-row tiles (W4A4), ragged tails included.
+@pytest.mark.parametrize("mode,T,E,k", [(mx.W4A16, 1300, 4, 2), (mx.W4A16, 1000, 3, 1),
                                         (mx.W4A4, 600, 4, 2), (mx.W4A4, 700, 5, 3)])
 def test_moe_large_token_tiles_all_tokens(mode, T, E, k):
     L = Layer(_small(T, 128, 192, E, k, seed=T + E + k))
     if mode == mx.W4A16:
-        assert _avg_rows(T, E, k) >= 320
+        assert mx.mxfp4_token_tile_rows(T * k, E, mode) == 192
         assert_close_tol(L.gpu(mode), L.ref(), what=f"moe T={T} E={E} k={k} W4A16 (192-row tiles)")
     else:
-        assert _avg_rows(T, E, k) > 64
+        assert mx.mxfp4_token_tile_rows(T * k, E, mode) == 128
         L.check_w4a4(what=f"moe T={T} E={E} k={k} W4A4 (128-row tiles)")
 
 
