@@ -222,7 +222,9 @@ MXFP4_API size_t moe_mxfp4_experts_workspace_size(int64_t P, int64_t H, int64_t 
                                                   mxfp4_mode mode);
 /* moe_mxfp4_combine: out[t] = bf16( sum_j y_sorted[inv[t*top_k + j]] ) summed in fp32 in
  * slot order j = 0 .. top_k-1 (deterministic); y_sorted fp32 [*, H], inv int32
- * [T*top_k], out bf16 [T, H].  Requires H % 8 == 0, top_k <= 8. */
+ * [T*top_k], out bf16 [T, H].  Requires H % 8 == 0, top_k <= 8.  The sum is the
+ * weighted combine of moe_mxfp4_mlp (the reading of "out = sum of weight x
+ * down(h)"; the routing weight is already in y). */
 MXFP4_API mxfp4_status moe_mxfp4_combine(const float* y_sorted, const int32_t* inv, int64_t T,
                                          int32_t top_k, int64_t H, void* out_bf16, void* stream);
 
@@ -271,7 +273,8 @@ MXFP4_API mxfp4_status moe_mxfp4_mlp_noalloc(const void* x_bf16, int64_t T, int6
                                              mxfp4_mode mode, void* stream);
 
 /* ---------------------------------------------------------------- tracing
- * Optional stage timing for the calling host thread.  `events` points to
+ * Optional stage timing for the calling host thread (no counterpart in the pages:
+ * the benchmark's per-stage timing).  `events` points to
  * `n_events` cudaEvent_t handles (passed as void*) created by the caller; while
  * set, moe_mxfp4_mlp records events[i] on its stream at stage boundary i:
  *   0 start, 1 after routing + gather (W4A4: + activation quantization),
@@ -282,6 +285,7 @@ MXFP4_API mxfp4_status moe_mxfp4_mlp_noalloc(const void* x_bf16, int64_t T, int6
 MXFP4_API void mxfp4_set_trace_events(void* const* events, int n_events);
 
 /* ---------------------------------------------------------------- status
+ * Error reporting (no counterpart in the pages).
  * Synchronizes `stream`, then returns and clears the current device's device-side
  * status word (MXFP4_OK, or MXFP4_ERR_TIMEOUT if a kernel gave up waiting).
  * Returns MXFP4_ERR_CUDA if the synchronization itself failed. */
