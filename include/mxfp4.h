@@ -119,8 +119,8 @@ MXFP4_API size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp
  * the MoE layer (rows = T * top_k).  W4A16: 16, 32, 64, 128 or 192, the size with the
  * least measured tile cost times tiles for a group one standard deviation above the
  * mean; W4A4: the smallest of 16, 32, 64, 128 that holds the mean.  A host query for
- * tests and tuning: no CUDA call.  Returns 0 when rows < 1, groups < 1 or the mode is
- * unknown.  No counterpart in the pages: the launch policy of the GEMMs above. */
+ * tests and tuning: no CUDA call.  Returns 0 when rows or groups is below 1 or at
+ * least 2^62, or the mode is unknown.  No counterpart in the pages: the launch policy of the GEMMs above. */
 MXFP4_API int32_t mxfp4_token_tile_rows(int64_t rows, int64_t groups, mxfp4_mode mode);
 
 /* ---------------------------------------------------------------- routing

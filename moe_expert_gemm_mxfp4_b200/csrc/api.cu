@@ -439,7 +439,7 @@ size_t mxfp4_gemm_workspace_size(int64_t M, int64_t K, int64_t N, mxfp4_mode mod
 }
 
 int32_t mxfp4_token_tile_rows(int64_t rows, int64_t groups, mxfp4_mode mode) {
-    if (rows < 1 || groups < 1) return 0;
+    if (rows < 1 || groups < 1 || rows >= (int64_t{1} << 62) || groups >= (int64_t{1} << 62)) return 0;
     if (mode == MXFP4_W4A16) return mx::pick_token_tiling(rows, groups).nt;
     if (mode == MXFP4_W4A4) return mx::pick_token_tiling_w4a4(rows, groups).nt;
     return 0;

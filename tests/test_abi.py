@@ -101,6 +101,8 @@ def test_w4a4_token_tiles_and_invalid_queries(lib):
     assert lib.mxfp4_token_tile_rows(0, 1, 0) == 0
     assert lib.mxfp4_token_tile_rows(8, 0, 0) == 0
     assert lib.mxfp4_token_tile_rows(8, 1, 7) == 0
+    assert lib.mxfp4_token_tile_rows(1 << 62, 1, 0) == 0          # no overflow in the mean
+    assert lib.mxfp4_token_tile_rows((1 << 62) - 1, 1 << 40, 0) == 192
 
 
 def test_route_and_moe_argument_checks(lib):
